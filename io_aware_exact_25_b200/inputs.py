@@ -1,0 +1,100 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module draws random numbers and rounds them to bf16; it holds none of
+the attention arithmetic.  Both the CUDA path and the fp64 oracle consume the
+same bf16 tensors it returns.
+
+Recipe (the same for every workload):
+  * ``g = torch.Generator().manual_seed(seed)`` on the CPU;
+  * draw fp32 ``randn`` tensors of shape ``[B, H, N, d]`` in the order
+    Q, K, V, dO;
+  * ``qkv_scale`` multiplies Q, K and V (exact for 0.5);
+  * ``offset_norm > 0``: draw ``g_h ~ N(0, I_d)`` per head (after dO), set
+    ``u_h = offset_norm * g_h / |g_h|`` and add the same ``u_h`` to every row
+    of both Q and K of head h (peaked softmax rows);
+  * round each tensor to bf16 (round-to-nearest-even).
+
+The named workloads stand in for the pages' model-level benchmarks (BERT,
+GPT-3, ViT at sequence lengths 512-2048, and the 32K/64K long-context
+examples), none of which can be reproduced without models or data.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    p_drop: float
+    seed: int
+    qkv_scale: float = 1.0
+    offset_norm: float = 0.0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def fwd_flops(self) -> float:
+        """4*B*H*N^2*d, halved when causal (the attention FLOP convention)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2.0 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        """2.5x the forward (five GEMMs against two)."""
+        return 2.5 * self.fwd_flops()
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 2, 128, 64, False, 0.0, 0),
+    "train2k": Workload("train2k", 4, 16, 2048, 64, False, 0.0, 1),
+    "train2k_causal": Workload("train2k_causal", 4, 16, 2048, 64, True, 0.0, 1),
+    "long8k_causal": Workload("long8k_causal", 2, 16, 8192, 128, True, 0.0, 2, qkv_scale=0.5),
+    "long32k_causal": Workload("long32k_causal", 1, 16, 32768, 128, True, 0.0, 3, offset_norm=2.0),
+    "long64k_causal_dropout": Workload("long64k_causal_dropout", 1, 8, 65536, 128, True, 0.1, 4),
+}
+
+
+def make_inputs(B: int, H: int, N: int, d: int, seed: int, qkv_scale: float = 1.0,
+                offset_norm: float = 0.0) -> dict:
+    """Return ``{'q','k','v','do'}`` as contiguous bf16 CPU tensors ``[B,H,N,d]``."""
+    g = torch.Generator().manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    do = torch.randn(shape, generator=g, dtype=torch.float32)
+    if qkv_scale != 1.0:
+        q.mul_(qkv_scale)
+        k.mul_(qkv_scale)
+        v.mul_(qkv_scale)
+    if offset_norm > 0.0:
+        gh = torch.randn((H, d), generator=g, dtype=torch.float32)
+        u = offset_norm * gh / gh.norm(dim=-1, keepdim=True)
+        q.add_(u.view(1, H, 1, d))
+        k.add_(u.view(1, H, 1, d))
+    return {n: t.to(torch.bfloat16).contiguous() for n, t in
+            (("q", q), ("k", k), ("v", v), ("do", do))}
+
+
+def workload_inputs(w: Workload) -> dict:
+    return make_inputs(w.B, w.H, w.N, w.d, w.seed, w.qkv_scale, w.offset_norm)
+
+
+def sample_rows(N: int, count: int, seed: int) -> list:
+    """Sorted sample of ``count`` distinct rows of ``range(N)`` that always
+    contains 0 and N-1, drawn from a generator seeded with ``1000 + seed``."""
+    if count >= N:
+        return list(range(N))
+    g = torch.Generator().manual_seed(1000 + int(seed))
+    perm = torch.randperm(N - 2, generator=g)[: max(0, count - 2)] + 1
+    rows = sorted(set([0, N - 1] + perm.tolist()))
+    return rows

@@ -1,0 +1,49 @@
+"""The oracle pins must catch plausible mistakes in the oracle.
+
+Each case compiles a copy of ``oracle/attention_oracle.c`` with one planted
+mistake (a dropped term, a wrong sign or index, a transposed operand, a wrong
+dropout scale ...) and runs the pin suite against it in a subprocess; the
+suite has to fail.  Mistakes are planted only in the oracle, on the CPU.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
+
+MUTANTS = {
+    "drop_minus_D_in_dS": ("double ds = p * (dp - D);", "double ds = p * dp;"),
+    "causal_mask_transposed": ("if (pb->causal && j > i) {", "if (pb->causal && j < i) {"),
+    "causal_mask_off_by_one": ("if (pb->causal && j > i) {", "if (pb->causal && j >= i) {"),
+    "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "dropout_scale_inverted": ("const double inv_keep = 1.0 / (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;",
+                               "const double inv_keep = (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;"),
+    "dq_missing_scale": ("for (int c = 0; c < pb->d; ++c) dq[c] *= pb->scale;", ""),
+    "dk_uses_k_not_q": ("dkj[c] += ds * elem(qi, c);", "dkj[c] += ds * elem(kj, c);"),
+    "dv_without_dropout_mask": ("double pd = p * z;", "double pd = p;"),
+    "softmax_not_normalised": ("static double prob(double s, double m, double l) { return exp(s - m) / l; }",
+                               "static double prob(double s, double m, double l) { (void)l; return exp(s - m); }"),
+    "hash_constant_typo": ("C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32);",
+                           "C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32) + 2u;"),
+    "threshold_floor": ("double t = ceil(p * 4294967296.0);", "double t = floor(p * 4294967296.0);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    before, after = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(before) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(text.replace(before, after))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", str(so),
+                    str(mutant_c), "-lm"], check=True)
+    env = dict(os.environ, ORACLE_LIB=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
