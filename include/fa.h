@@ -1,0 +1,128 @@
+/*
+ * fa.h -- C ABI of the sm_100a fused exact-attention library (libfa_sm100.so).
+ *
+ * Exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * ("FlashAttention for Efficient Training", section 1, attention equation),
+ * computed by one fused, tiled forward kernel with an online softmax that
+ * saves the per-row logsumexp ("How FlashAttention Optimizes GPU Memory for
+ * Fast AI Training": Tiling, Online Softmax, Kernel Fusion; "FlashAttention
+ * for Efficient Training" section 3.2, log_softmax / logsumexp), and a fused
+ * backward that recomputes S and P tile by tile from Q, K, V and the saved
+ * logsumexp ("How FlashAttention Optimizes GPU Memory for Fast AI Training",
+ * Recomputation in the Backward Pass; "FlashAttention for Efficient
+ * Training" section 3.2, dV = P^T dO, and the chain rule for dQ, dK).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are dense, contiguous, row-major [B, H, N, d] arrays of bf16
+ *    (IEEE bfloat16 bit patterns) in device memory, 16-byte aligned.
+ *    lse and the backward's D are fp32 [B, H, N] in device memory.
+ *  - d (head dimension) is 64 or 128.  N >= 1 is any length; B, H >= 1.
+ *    B = 0, H = 0 or N = 0 is an empty problem: the call returns FA_OK and
+ *    launches nothing (pointers are then not inspected).
+ *  - scale > 0 and finite (1/sqrt(d) is the usual choice).  causal is 0 or 1:
+ *    query i sees keys j <= i.  dropout_p in [0, 1): element (i, j) of head
+ *    (b, h) is kept iff hash32(seed, b, h, i, j) >= ceil(dropout_p * 2^32)
+ *    (hash32 is defined in io_aware_exact_25_b200/csrc/dropout_hash.cuh);
+ *    kept probabilities are scaled by 1/(1-p).
+ *    Dropout is applied after the softmax, so lse is that of the undropped
+ *    scores.  The backward with the same (seed, dropout_p) regenerates the
+ *    same mask.
+ *  - The caller owns every buffer.  The library allocates no device or host
+ *    memory; it keeps one device-resident error word per device.
+ *  - stream is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream; nothing synchronises.
+ *  - On any error nothing is launched and a negative fa_status is returned.
+ *    Calls are thread-safe.
+ */
+#ifndef FA_SM100_H_
+#define FA_SM100_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad scale/causal/p */
+  FA_ERR_UNSUPPORTED = -2, /* head dimension other than 64 or 128 */
+  FA_ERR_ALIGNMENT = -3,   /* a tensor not 16-byte aligned (lse/D: 4-byte) */
+  FA_ERR_WORKSPACE = -4,   /* workspace null or smaller than required */
+  FA_ERR_CUDA = -5,        /* a CUDA runtime/driver call or launch failed */
+  FA_ERR_DEVICE = -6,      /* a kernel reported an error (fa_get_device_error) */
+  FA_ERR_TOO_LARGE = -7    /* sizes overflow the library's index range */
+} fa_status;
+
+/*
+ * Forward ("FlashAttention for Efficient Training" section 3, Workflow
+ * Breakdown steps 1-3: block loading, local attention with the online
+ * softmax, incremental output accumulation; fused scaling, masking and
+ * dropout per section 3, Fused Kernel Design).  Reads q, k, v [B,H,N,d]
+ * bf16; writes o [B,H,N,d] bf16 and lse [B,H,N] fp32 (natural-log logsumexp
+ * of scale * q_i . k_j over the visible keys j).  o and lse must not alias
+ * the inputs.  Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED,
+ * FA_ERR_ALIGNMENT, FA_ERR_TOO_LARGE (nothing launched) or FA_ERR_CUDA.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, float dropout_p, uint64_t seed, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for this shape: an fp32 dQ
+ * accumulator [B,H,N,d] plus two fp32 row vectors (scaled lse and
+ * D_i = dO_i . O_i) padded to a multiple of 128 rows.  Returns 0 for an empty
+ * problem or invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward with recomputation ("FlashAttention for Efficient Training"
+ * section 3.2, Integration with Autograd Engines: dV = P^T dO, dQ and dK by
+ * the chain rule; "How FlashAttention Optimizes GPU Memory for Fast AI
+ * Training", Recomputation in the Backward Pass).  Three launches on
+ * `stream`: a row pass (D_i = dO_i . O_i, scaled lse, zeroed dQ accumulator),
+ * the fused recompute kernel, and the dQ conversion.  Reads q, k, v, o, dout [B,H,N,d] bf16 and lse [B,H,N] fp32
+ * from fa_fwd with the same scale/causal/dropout_p/seed; writes dq, dk, dv
+ * [B,H,N,d] bf16.  workspace (16-byte aligned, at least
+ * fa_bwd_workspace_size bytes) is scratch owned by the caller; its contents
+ * on entry do not matter.  dq/dk/dv must not alias any input.
+ * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.  dQ is accumulated in fp32 with atomic adds, so its bits may differ from run
+ * to run by rounding order; dK and dV are deterministic.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p,
+           uint64_t seed, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Debug export of the dropout mask: for each listed head bh = b*H + h
+ * (heads[nheads]) and query row (rows[nrows]), writes the keep bit of every
+ * key j < N to out[(hi * nrows + ri) * N + j] (1 = kept).  heads, rows and
+ * out are device pointers.  Uses the same device hash the kernels inline.
+ */
+int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,
+                    const int32_t* rows, int nrows, uint8_t* out, void* stream);
+
+/* Static description of a status code. */
+const char* fa_strerror(int status);
+
+/* The cudaError_t of the most recent FA_ERR_CUDA on this thread (0 if none). */
+int fa_last_cuda_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error
+ * word.  Returns 0 if no kernel reported an error since the last read, else
+ * the kernel's code (1 = a bounded wait timed out, 2 = shared memory
+ * misaligned); FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_get_device_error(void* stream);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H_ */

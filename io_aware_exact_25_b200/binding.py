@@ -1,0 +1,154 @@
+"""Thin ctypes binding over the C ABI in ``include/fa.h``.
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels of ``libfa_sm100.so``.  Tensors are torch CUDA tensors (torch supplies
+device memory and the current stream); outputs are allocated here with torch
+when the caller does not pass them.  There is no CPU fallback: a missing
+library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_ALIGNMENT = -3
+FA_ERR_WORKSPACE = -4
+FA_ERR_CUDA = -5
+FA_ERR_DEVICE = -6
+FA_ERR_TOO_LARGE = -7
+
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_dropout_mask", "fa_strerror",
+           "fa_last_cuda_error", "fa_get_device_error", "fa_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {strerror(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load ``libfa_sm100.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; build it with "
+                               "io_aware_exact_25_b200.build.build()")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, I, F, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
+        lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
+        lib.fa_bwd_workspace_size.restype = SZ
+        lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
+        lib.fa_strerror.argtypes = [I]
+        lib.fa_strerror.restype = ctypes.c_char_p
+        lib.fa_get_device_error.argtypes = [vp]
+        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_dropout_mask, lib.fa_get_device_error,
+                   lib.fa_last_cuda_error, lib.fa_version):
+            fn.restype = I
+        _lib = lib
+        return lib
+
+
+def strerror(status: int) -> str:
+    return load().fa_strerror(int(status)).decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (there is no CPU path)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v, o, dO must be bf16")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B,H,N,d]")
+        if t.dim() != 4:
+            raise ValueError("tensors must be [B,H,N,d]")
+
+
+def _call(rc: int, what: str):
+    if rc != FA_OK:
+        raise FaError(rc, what)
+
+
+def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=None, stream=None):
+    """O and lse of exact attention via ``fa_fwd``."""
+    _check_inputs(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                       int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
+    _call(rc, "fa_fwd")
+    return o, lse
+
+
+def bwd_workspace_size(B, H, N, d) -> int:
+    return int(load().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, dq=None, dk=None,
+        dv=None, workspace=None, stream=None):
+    """dQ, dK, dV via ``fa_bwd`` (allocates the workspace with torch if not given)."""
+    _check_inputs(q, k, v, o, dout)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                       _ptr(dv), B, H, N, d, float(scale), int(bool(causal)), float(dropout_p), int(seed),
+                       _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                       _stream(stream))
+    _call(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def dropout_mask(B, H, N, dropout_p, seed, heads, rows, device="cuda", stream=None):
+    """Keep bits [nheads, nrows, N] (uint8) from the device hash."""
+    h = torch.as_tensor(heads, dtype=torch.int32, device=device).contiguous()
+    r = torch.as_tensor(rows, dtype=torch.int32, device=device).contiguous()
+    out = torch.empty((h.numel(), r.numel(), N), dtype=torch.uint8, device=device)
+    rc = load().fa_dropout_mask(B, H, N, float(dropout_p), int(seed), _ptr(h), h.numel(), _ptr(r),
+                                r.numel(), _ptr(out), _stream(stream))
+    _call(rc, "fa_dropout_mask")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the kernels' error word."""
+    return int(load().fa_get_device_error(_stream(stream)))

@@ -1,0 +1,617 @@
+// bwd_sm100.cuh -- fused attention backward for sm_100a.
+//
+// Recomputes S and P tile by tile from Q, K, V and the saved logsumexp
+// instead of storing them ("How FlashAttention Optimizes GPU Memory for Fast
+// AI Training", Recomputation in the Backward Pass; "FlashAttention for
+// Efficient Training" section 2, Forward Pass with Recomputation).  With
+// Pd = P * Z / (1 - p) the dropped probabilities (Z the keep mask):
+//   dV = Pd^T dO                 ("FlashAttention for Efficient Training",
+//                                 section 3.2, Integration with Autograd)
+//   dP = (dO V^T) * Z / (1 - p)
+//   D_i = sum_j P_ij dP_ij = dO_i . O_i
+//   dS = P * (dP - D)
+//   dQ = scale * dS K,  dK = scale * dS^T Q      (chain rule)
+// The pages' printed dQ formulas are garbled; the expressions above follow
+// from the attention definition and are what the fp64 oracle checks.
+//
+// Three launches:
+//  1. row pass: D_i = dO_i . O_i and lse2_i = lse_i * log2(e) per row (rows
+//     padded to a multiple of 128 get lse2 = +inf so their P is 0), and a
+//     zeroed fp32 dQ accumulator;
+//  2. the fused recompute kernel, one CTA per 128-key tile K_j, V_j of a
+//     head, looping over the 128-row query tiles i that see it (i >= j when
+//     causal).  Per step it computes, in tensor memory with keys on the lanes,
+//     S^T = K_j Q_i^T and dP^T = V_j dO_i^T, forms P^T and dS^T in registers,
+//     accumulates dV += P^T dO_i and dK += dS^T Q_i in tensor memory, and
+//     computes the dQ_i partial dS K_j, which a warpgroup adds into the fp32
+//     accumulator with vector atomics (red.global.add.v4.f32);
+//  3. dQ = scale * accumulator, rounded to bf16.
+// Warp roles of the fused kernel:
+//   warps 0-3   P/dS for query columns 0-63 of the step   (TMEM lanes = keys)
+//   warps 4-7   P/dS for query columns 64-127
+//   warps 8-11  dQ read-out and atomic accumulation        (TMEM lanes = queries)
+//   warp  12    tcgen05 MMA issue (one thread)
+//   warp  13    TMA producer (+ dropout row keys)
+// Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
+// [0,32) and [64,96); R_dP [128,256) dP^T fp32, then dS^T bf16 in [128,160)
+// and [192,224), then the dQ partial (fp32, D columns); dV at 256, dK at
+// 256 + D.  MMA order per step: dP(i), dV(i), dK(i), S(i+1), dQ(i), so the
+// next step's softmax overlaps this step's dQ read-out.
+#pragma once
+
+#include "dropout_hash.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+struct BwdArgs {
+  int B, H, N;
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  uint32_t drop_threshold;
+  float drop_scale;
+  uint64_t seed;
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* dout;
+  const float* lse;  // [BH, N] natural log
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dq_acc;  // [BH, N, D] fp32 scratch
+  float* lse2;    // [BH, Npad] scratch: lse * log2(e), +inf on padded rows
+  float* drow;    // [BH, Npad] scratch: D_i, 0 on padded rows
+  int* err;
+};
+
+__host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline size_t bwd_workspace_bytes(int BH, int N, int d) {
+  const size_t npad = round_up((size_t)N, 128);
+  return round_up((size_t)BH * N * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256);
+}
+
+inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, float** lse2, float** drow) {
+  const size_t npad = round_up((size_t)N, 128);
+  char* p = static_cast<char*>(ws);
+  *dq_acc = reinterpret_cast<float*>(p);
+  p += round_up((size_t)BH * N * d * 4, 256);
+  *lse2 = reinterpret_cast<float*>(p);
+  p += round_up((size_t)BH * npad * 4, 256);
+  *drow = reinterpret_cast<float*>(p);
+}
+
+// ------------------------------------------------------------ row pass
+
+// One warp per (padded) row: D_i = sum_c dO_ic O_ic in fp32, lse2_i, and the
+// row of the dQ accumulator set to zero.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, int npad) {
+  constexpr int kPer = D / 32;  // elements per lane
+  const long long rows = (long long)BH * npad;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r = warp0; r < rows; r += nwarps) {
+    const int bh = (int)(r / npad);
+    const int i = (int)(r - (long long)bh * npad);
+    if (i < a.N) {
+      const size_t off = ((size_t)bh * a.N + i) * D + lane * kPer;
+      float acc = 0.f;
+      if (kPer == 4) {
+        const uint2 ov = *reinterpret_cast<const uint2*>(a.o + off);
+        const uint2 dv = *reinterpret_cast<const uint2*>(a.dout + off);
+        acc = bf16_lo(ov.x) * bf16_lo(dv.x) + bf16_hi(ov.x) * bf16_hi(dv.x) + bf16_lo(ov.y) * bf16_lo(dv.y) +
+              bf16_hi(ov.y) * bf16_hi(dv.y);
+        *reinterpret_cast<float4*>(a.dq_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const uint32_t ov = *reinterpret_cast<const uint32_t*>(a.o + off);
+        const uint32_t dv = *reinterpret_cast<const uint32_t*>(a.dout + off);
+        acc = bf16_lo(ov) * bf16_lo(dv) + bf16_hi(ov) * bf16_hi(dv);
+        *reinterpret_cast<float2*>(a.dq_acc + off) = make_float2(0.f, 0.f);
+      }
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+      if (lane == 0) {
+        a.drow[r] = acc;
+        a.lse2[r] = a.lse[(size_t)bh * a.N + i] * 1.4426950408889634f;
+      }
+    } else if (lane == 0) {
+      a.drow[r] = 0.f;
+      a.lse2[r] = INFINITY;
+    }
+  }
+}
+
+// dQ = scale * accumulator, 8 elements per thread per iteration.
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                       long long n8, float scale) {
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n8;
+       u += (long long)gridDim.x * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[2 * u];
+    const float4 y = reinterpret_cast<const float4*>(acc)[2 * u + 1];
+    uint4 w;
+    w.x = pack_bf16x2(x.x * scale, x.y * scale);
+    w.y = pack_bf16x2(x.z * scale, x.w * scale);
+    w.z = pack_bf16x2(y.x * scale, y.y * scale);
+    w.w = pack_bf16x2(y.z * scale, y.w * scale);
+    reinterpret_cast<uint4*>(dq)[u] = w;
+  }
+}
+
+// ------------------------------------------------------- fused kernel
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kThreads = 448;
+  static constexpr uint32_t kHalf = 128u * 128u;
+  static constexpr uint32_t kTile = 128u * D * 2u;
+  static constexpr int kQStages = 2;
+  static constexpr int kDoStages = D == 128 ? 1 : 2;
+  static constexpr uint32_t kOffK = 0;
+  static constexpr uint32_t kOffV = kOffK + kTile;
+  static constexpr uint32_t kOffQ = kOffV + kTile;
+  static constexpr uint32_t kOffDO = kOffQ + kQStages * kTile;
+  static constexpr uint32_t kOffDS = kOffDO + kDoStages * kTile;  // dS, 128 x 128 bf16, MN-major halves
+  static constexpr uint32_t kRowStage = 3u * 128u * 4u;             // lse2, D, dropout row keys
+  static constexpr uint32_t kOffRow = kOffDS + 2u * kHalf;
+  static constexpr uint32_t kOffBar = kOffRow + 2u * kRowStage;
+  // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
+  // row_empty[2], s, dp, p, ds, dv, dk, dq, dq_free, drain
+  static constexpr int kNumBars = 1 + 12 + 9;
+  static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+// TMEM column of the packed bf16 operand slice kk (16 queries) written by the
+// two P/dS warpgroups: queries 0-63 at [0,32), 64-127 at [64,96).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
+
+template <int D, bool CAUSAL, bool DROPOUT>
+__global__ void __launch_bounds__(448, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdArgs a) {
+  using L = BwdLayout<D>;
+  static_assert(D == 64 || D == 128, "head dim");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* bar_kv = bars;
+  uint64_t* bar_q_full = bars + 1;
+  uint64_t* bar_q_empty = bars + 3;
+  uint64_t* bar_do_full = bars + 5;
+  uint64_t* bar_do_empty = bars + 7;
+  uint64_t* bar_row_full = bars + 9;
+  uint64_t* bar_row_empty = bars + 11;
+  uint64_t* bar_s = bars + 13;
+  uint64_t* bar_dp = bars + 14;
+  uint64_t* bar_p = bars + 15;
+  uint64_t* bar_ds = bars + 16;
+  uint64_t* bar_dv = bars + 17;
+  uint64_t* bar_dk = bars + 18;
+  uint64_t* bar_dq = bars + 19;
+  uint64_t* bar_dq_free = bars + 20;
+  uint64_t* bar_drain = bars + 21;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int BH = a.B * a.H;
+  const int nT = (a.N + 127) >> 7;
+  const int jt = blockIdx.x / BH;  // key tile; ascending = most query tiles first when causal
+  const int bh = blockIdx.x - jt * BH;
+  const int i_begin = CAUSAL ? jt : 0;
+  const int n_steps = nT - i_begin;
+  const int npad = nT * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_q_full[s], 1);
+      mbar_init(&bar_q_empty[s], 1);
+      mbar_init(&bar_do_full[s], 1);
+      mbar_init(&bar_do_empty[s], 1);
+      mbar_init(&bar_row_full[s], 1);
+      mbar_init(&bar_row_empty[s], 256);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
+    mbar_init(bar_dv, 1);
+    mbar_init(bar_dk, 1);
+    mbar_init(bar_dq, 1);
+    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_drain, 1);
+    const bool misaligned = (sbase & 1023u) != 0u;
+    *abort_flag = misaligned ? 1 : 0;
+    if (misaligned && a.err) atomicCAS(a.err, kDevOk, kDevMisaligned);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, a.err};
+  const bool run = *abort_flag == 0;
+
+  if (run && warp == 13) {
+    // ------------------------------------------------------ TMA producer
+    const uint64_t pol_keep = policy_evict_last();
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_3d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, bh, bar_kv, pol_keep);
+        tma_load_3d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, jt * 128, bh, bar_kv, pol_keep);
+      }
+    }
+    // All 32 lanes run this loop (they compute the dropout row keys); the
+    // waits are made warp-uniform with __all_sync, lane 0 issues the copies.
+    int q_issued = 0, do_issued = 0;
+    bool ok = true;
+    for (int it = 0; it < n_steps && ok; ++it) {
+      const int i = i_begin + it;
+      // Q_i and dO_i: re-read by every key tile of the head -> keep in L2
+      const int qs = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_q_empty[qs], ((it >> 1) & 1) ^ 1u, ab))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, bh,
+                      &bar_q_full[qs], pol_keep);
+      }
+      ++q_issued;
+      const int ds_ = it % L::kDoStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_do_empty[ds_], ((it / L::kDoStages) & 1) ^ 1u, ab))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_do_full[ds_], L::kTile);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, bh,
+                      &bar_do_full[ds_], pol_keep);
+      }
+      ++do_issued;
+      // row statistics of query tile i
+      const int rs = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_row_empty[rs], ((it >> 1) & 1) ^ 1u, ab))) {
+        ok = false;
+        break;
+      }
+      uint8_t* rowbuf = smem + L::kOffRow + rs * L::kRowStage;
+      if (DROPOUT) {
+        uint32_t* keys = reinterpret_cast<uint32_t*>(rowbuf + 2 * 512);
+        for (int c = lane; c < 128; c += 32)
+          keys[c] = dropout_row_key(a.seed, (uint32_t)(bh / a.H), (uint32_t)(bh % a.H), (uint32_t)(i * 128 + c));
+        __syncwarp();
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_row_full[rs], 1024);
+        bulk_load(rowbuf, a.lse2 + (size_t)bh * npad + i * 128, 512, &bar_row_full[rs]);
+        bulk_load(rowbuf + 512, a.drow + (size_t)bh * npad + i * 128, 512, &bar_row_full[rs]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      // Every load issued must land before the CTA may exit.
+      mbar_wait_drain(bar_kv, 0);
+      for (int n = q_issued > 2 ? q_issued - 2 : 0; n < q_issued; ++n) mbar_wait_drain(&bar_q_full[n & 1], (n >> 1) & 1);
+      for (int n = do_issued > L::kDoStages ? do_issued - L::kDoStages : 0; n < do_issued; ++n)
+        mbar_wait_drain(&bar_do_full[n % L::kDoStages], (n / L::kDoStages) & 1);
+    }
+  } else if (run && warp == 12) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdKK = idesc_bf16(128, 128, false, false);  // S^T, dP^T: both operands K-major
+      constexpr uint32_t kIdTM = idesc_bf16(128, D, false, true);     // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t kIdMM = idesc_bf16(128, D, true, true);      // dQ: both MN-major
+      const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sDS = sbase + L::kOffDS;
+      bool ok = mbar_wait(bar_kv, 0, ab) && mbar_wait(&bar_q_full[0], 0, ab);
+      bool issued_any = false;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t sQ0 = sbase + L::kOffQ;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQ0, kk, L::kHalf), kIdKK,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar_s);
+        issued_any = true;
+      }
+      for (int it = 0; it < n_steps && ok; ++it) {
+        const uint32_t ph = it & 1;
+        const int qs = it & 1;
+        const int ds_ = it % L::kDoStages;
+        const uint32_t sQ = sbase + L::kOffQ + qs * L::kTile;
+        const uint32_t sDO = sbase + L::kOffDO + ds_ * L::kTile;
+        // dP^T = V dO_i^T into R_dP (holds the previous dQ partial until read out)
+        if (!mbar_wait(&bar_do_full[ds_], (it / L::kDoStages) & 1, ab)) break;
+        if (it > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + L::kColDP, desc_kmajor(sV, kk, L::kHalf), desc_kmajor(sDO, kk, L::kHalf), kIdKK,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar_dp);
+        // dV += P^T dO_i
+        if (!mbar_wait(bar_p, ph, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::kColDV, tmem + L::kColS + packed_col(kk), desc_mnmajor(sDO, kk, L::kHalf), kIdTM,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_dv);
+        mma_commit(&bar_do_empty[ds_]);
+        // dK += dS^T Q_i
+        if (!mbar_wait(bar_ds, ph, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::kColDK, tmem + L::kColDP + packed_col(kk), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_dk);
+        mma_commit(&bar_q_empty[qs]);
+        // S^T for the next step, once dV has consumed P^T from R_S
+        if (it + 1 < n_steps) {
+          const int qn = (it + 1) & 1;
+          if (!mbar_wait(&bar_q_full[qn], ((it + 1) >> 1) & 1, ab)) break;
+          if (!mbar_wait(bar_dv, ph, ab)) break;
+          tc_fence_after();
+          const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQn, kk, L::kHalf), kIdKK,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_s);
+        }
+        // dQ_i partial = dS K_j into R_dP, once dK has consumed dS^T
+        if (!mbar_wait(bar_dk, ph, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar_dq);
+      }
+      if (issued_any) {
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else if (run && warp >= 8 && warp < 12) {
+    // ------------------------------------------ dQ read-out + accumulate
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // query within the tile == TMEM lane
+    const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDP;
+    for (int it = 0; it < n_steps; ++it) {
+      if (!mbar_wait(bar_dq, it & 1, ab)) break;
+      tc_fence_after();
+      const int q_row = (i_begin + it) * 128 + row;
+      float* dst = a.dq_acc + ((size_t)bh * a.N + (size_t)(q_row < a.N ? q_row : 0)) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t v[32];
+        tmem_ld32_sync(tQ + 32u * c4, v);
+        if (c4 == D / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar_dq_free);
+        }
+        if (q_row < a.N) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            red_add_v4(dst + 32 * c4 + 4 * k, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+        }
+      }
+    }
+  } else if (run && warp < 8) {
+    // --------------------------------------------------------- P and dS
+    const int wg = warp >> 2;
+    const int quad = warp & 3;
+    const int jr = quad * 32 + lane;  // key within the tile == TMEM lane
+    const int key = jt * 128 + jr;
+    const int col0 = 64 * wg;         // this warpgroup's query columns
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::kColS + col0;
+    const uint32_t tDP = tmem + lane_off + L::kColDP + col0;
+    const uint32_t tPst = tmem + lane_off + L::kColS + 64u * wg;   // packed P^T (32 columns)
+    const uint32_t tDSst = tmem + lane_off + L::kColDP + 64u * wg; // packed dS^T
+    const uint32_t sDSrow = sbase + L::kOffDS + wg * L::kHalf + jr * 128;
+    const float sl2 = a.scale_log2;
+    const bool key_ok = key < a.N;
+    bool ok = true;
+    for (int it = 0; it < n_steps; ++it) {
+      const int i = i_begin + it;
+      const uint32_t ph = it & 1;
+      const int rs = it & 1;
+      const uint32_t rowbuf = sbase + L::kOffRow + rs * L::kRowStage;
+      if (!mbar_wait(bar_s, ph, ab) || !mbar_wait(&bar_row_full[rs], (it >> 1) & 1, ab)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t u[2][32];
+      tmem_ld32(tS, u[0]);
+      tmem_ld32(tS + 32u, u[1]);
+      tmem_ld_wait();
+      reg_fence(u[0]);
+      reg_fence(u[1]);
+      // P^T_jq = 2^(s * scale * log2 e - lse2_q); padded queries have lse2 = +inf
+      float p[64];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = ld_shared_f4(rowbuf + 4u * (col0 + 4 * c4));
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          p[c] = ex2(fmaf(__uint_as_float(u[c >> 5][c & 31]), sl2, -lv[e]));
+        }
+      }
+      if (!key_ok) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) p[c] = 0.f;
+      }
+      if (CAUSAL && i == jt) {
+        // diagonal tile: query 128 i + col0 + c sees key 128 i + jr iff col0 + c >= jr
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (col0 + c < jr) p[c] = 0.f;
+      }
+      uint32_t keep_bits[2] = {0xffffffffu, 0xffffffffu};
+      if (DROPOUT) {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 k4 = ld_shared_f4(rowbuf + 1024u + 4u * (col0 + 4 * c4));
+          const uint32_t kv[4] = {__float_as_uint(k4.x), __float_as_uint(k4.y), __float_as_uint(k4.z),
+                                  __float_as_uint(k4.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            if (dropout_hash(kv[e], (uint32_t)key) < a.drop_threshold) keep_bits[c >> 5] &= ~(1u << (c & 31));
+          }
+        }
+      }
+      {
+        uint32_t pk[2][16];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float p0 = p[2 * c], p1 = p[2 * c + 1];
+          if (DROPOUT) {
+            p0 = ((keep_bits[(2 * c) >> 5] >> ((2 * c) & 31)) & 1u) ? p0 * a.drop_scale : 0.f;
+            p1 = ((keep_bits[(2 * c + 1) >> 5] >> ((2 * c + 1) & 31)) & 1u) ? p1 * a.drop_scale : 0.f;
+          }
+          pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tPst, pk[0]);
+        tmem_st16(tPst + 16u, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p);
+      }
+      // dS^T = P^T * (dP^T * Z / (1 - p) - D), two 32-column halves
+      if (!mbar_wait(bar_dp, ph, ab)) {
+        ok = false;
+        break;
+      }
+      // the previous dQ partial read sDS; wait for it before overwriting
+      if (it > 0 && !mbar_wait(bar_dq, ph ^ 1u, ab)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t g[32];
+        tmem_ld32_sync(tDP + 32u * hf, g);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c2 = 0; c2 < 8; ++c2) {
+          const float4 d4 = ld_shared_f4(rowbuf + 512u + 4u * (col0 + 32 * hf + 4 * c2));
+          const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 32 * hf + 4 * c2 + e;
+            float dp = __uint_as_float(g[4 * c2 + e]);
+            if (DROPOUT) dp = ((keep_bits[c >> 5] >> (c & 31)) & 1u) ? dp * a.drop_scale : 0.f;
+            ds[e] = p[c] * (dp - dv[e]);
+          }
+          pk[2 * c2] = pack_bf16x2(ds[0], ds[1]);
+          pk[2 * c2 + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        tmem_st16(tDSst + 16u * hf, pk);
+        // shared-memory copy (A operand of dQ = dS K): row jr of this half,
+        // 16-byte chunks XOR-swizzled by (jr mod 8)
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint32_t chunk = (uint32_t)(4 * hf + q8);
+          st_shared_v4(sDSrow + ((chunk ^ (uint32_t)(jr & 7)) << 4), pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2],
+                       pk[4 * q8 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+      mbar_arrive(&bar_row_empty[rs]);
+    }
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK = scale * acc
+    if (ok && n_steps > 0 && mbar_wait(bar_dk, (n_steps - 1) & 1, ab)) {
+      tc_fence_after();
+      const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
+      const float mul = wg == 0 ? 1.f : a.scale;
+      __nv_bfloat16* dst = (wg == 0 ? a.dv : a.dk) + ((size_t)bh * a.N + (size_t)(key_ok ? key : 0)) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t v[32];
+        tmem_ld32_sync(src + 32u * c4, v);
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          w[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+        if (key_ok) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mdo, const BwdArgs& a, cudaStream_t st) {
+  using L = BwdLayout<D>;
+  auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
+  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mdo, const BwdArgs& a, bool causal, bool dropout, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  const int npad = (a.N + 127) / 128 * 128;
+  bwd_pre_kernel<D><<<148 * 8, 256, 0, st>>>(a, BH, npad);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (causal)
+    e = dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, a, st)
+                : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, a, st);
+  else
+    e = dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, a, st)
+                : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, a, st);
+  if (e != cudaSuccess) return e;
+  const long long n8 = (long long)BH * a.N * D / 8;
+  bwd_post_kernel<<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, n8, a.scale);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mdo, const BwdArgs& a, int d, bool causal, bool dropout,
+                              cudaStream_t st) {
+  return d == 64 ? launch_bwd_d<64>(mq, mk, mv, mdo, a, causal, dropout, st)
+                 : launch_bwd_d<128>(mq, mk, mv, mdo, a, causal, dropout, st);
+}
+
+}  // namespace fa

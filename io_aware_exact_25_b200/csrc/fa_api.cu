@@ -1,0 +1,256 @@
+// fa_api.cu -- host side of the C ABI declared in include/fa.h: argument
+// validation, TMA tensor-map construction, kernel selection and launch on
+// the caller's stream.  Allocates nothing; the only state is one device
+// error word per device (a __device__ variable in this module).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "bwd_sm100.cuh"
+#include "dropout_hash.cuh"
+#include "fwd_sm100.cuh"
+
+namespace {
+
+__device__ int g_device_error;  // kernels record kDevTimeout / kDevMisaligned here
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so the
+// library needs no link-time dependency on libcuda.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map of a [BH, N, d] bf16 tensor read in 128-row x 64-column boxes
+// with the 128-byte swizzle; rows past N read as zero.
+int make_tile_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2u, (cuuint64_t)N * (cuuint64_t)d * 2u};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
+int* device_error_ptr() {
+  int* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
+  return p;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shared argument checks.  Returns FA_OK, a negative status, or 1 for an
+// empty problem (nothing to do).
+int check_common(int B, int H, int N, int d, float scale, int causal, float dropout_p) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return 1;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long bh = (long long)B * H;
+  const long long elems = bh * (long long)N * d;
+  // grid sizes and 32-bit row counters stay in range
+  if (bh > (1ll << 24) || (long long)N > (1ll << 24) || elems > (1ll << 40)) return FA_ERR_TOO_LARGE;
+  if (bh * (((long long)N + 127) / 128) > 0x7fffffffll) return FA_ERR_TOO_LARGE;
+  return FA_OK;
+}
+
+uint32_t keep_threshold(float p) {
+  const double t = std::ceil((double)p * 4294967296.0);
+  if (t <= 0.0) return 0u;
+  if (t >= 4294967295.0) return 4294967295u;
+  return (uint32_t)t;
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+               cudaStream_t st) {
+  using L = fa::FwdLayout<D>;
+  auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const long long grid = (long long)a.B * a.H * ((a.N + 255) / 256);
+  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+template <int D>
+int dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+                 bool causal, bool dropout, cudaStream_t st) {
+  if (causal)
+    return dropout ? launch_fwd<D, true, true>(mq, mk, mv, a, st) : launch_fwd<D, true, false>(mq, mk, mv, a, st);
+  return dropout ? launch_fwd<D, false, true>(mq, mk, mv, a, st) : launch_fwd<D, false, false>(mq, mk, mv, a, st);
+}
+
+__global__ void dropout_mask_kernel(int H, int N, uint32_t threshold, uint64_t seed, const int32_t* heads,
+                                    int nheads, const int32_t* rows, int nrows, uint8_t* out) {
+  const long long total = (long long)nheads * nrows * N;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < total;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(u % N);
+    const long long hr = u / N;
+    const int ri = (int)(hr % nrows);
+    const int hi = (int)(hr / nrows);
+    const int bh = heads[hi];
+    const uint32_t key = fa::dropout_row_key(seed, (uint32_t)(bh / H), (uint32_t)(bh % H), (uint32_t)rows[ri]);
+    out[u] = fa::dropout_hash(key, (uint32_t)j) >= threshold ? 1 : 0;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_strerror(int status) {
+  switch (status) {
+    case FA_OK: return "success";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension (64 or 128)";
+    case FA_ERR_ALIGNMENT: return "tensor pointer misaligned (16 bytes; lse/D 4 bytes)";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA call failed (see fa_last_cuda_error)";
+    case FA_ERR_DEVICE: return "a kernel reported an error";
+    case FA_ERR_TOO_LARGE: return "problem too large for this library";
+    default: return "unknown status";
+  }
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int fa_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int value = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&value, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return value;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, float dropout_p, uint64_t seed, void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
+  fa::FwdArgs a;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.drop_threshold = keep_threshold(dropout_p);
+  a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
+  a.seed = seed;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.err = device_error_ptr();
+  if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
+  const bool dropout = dropout_p > 0.f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? dispatch_fwd<64>(mq, mk, mv, a, causal != 0, dropout, st)
+                 : dispatch_fwd<128>(mq, mk, mv, a, causal != 0, dropout, st);
+}
+
+int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,
+                    const int32_t* rows, int nrows, uint8_t* out, void* stream) {
+  if (B < 0 || H < 0 || N < 0 || nheads < 0 || nrows < 0) return FA_ERR_INVALID_ARG;
+  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0 || nheads == 0 || nrows == 0) return FA_OK;
+  if (!heads || !rows || !out) return FA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dropout_mask_kernel<<<1184, 256, 0, st>>>(H, N, keep_threshold(dropout_p), seed, heads, nheads, rows, nrows,
+                                             out);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.f, 0, 0.f) != FA_OK) return 0;
+  return fa::bwd_workspace_bytes(B * H, N, d);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p,
+           uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = fa::bwd_workspace_bytes(B * H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mdo, dout, B * H, N, d)) != FA_OK) return rc;
+  fa::BwdArgs a;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.drop_threshold = keep_threshold(dropout_p);
+  a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
+  a.seed = seed;
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.lse = lse;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  fa::bwd_workspace_split(workspace, B * H, N, d, &a.dq_acc, &a.lse2, &a.drow);
+  a.err = device_error_ptr();
+  if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fa::launch_bwd(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f, st);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,358 @@
+// fwd_sm100.cuh -- fused attention forward for sm_100a.
+//
+// O = softmax(scale * Q K^T [+ causal mask]) V with an optional dropout mask
+// applied to the probabilities, and lse = logsumexp of each (undropped,
+// scaled, masked) score row.  The method is the tiled, fused forward with an
+// online softmax: "How FlashAttention Optimizes GPU Memory for Fast AI
+// Training" (Tiling, Online Softmax, Kernel Fusion) and "FlashAttention for
+// Efficient Training" section 3 (Algorithmic Details: S_ij = Q_i K_j^T /
+// sqrt(d_k) per block, running maxima and sums, O written once) and
+// section 3.2 (logsumexp, rescaling during accumulation).
+//
+// One CTA owns 256 query rows of one head as two 128-row tiles Q0, Q1 and
+// streams 128-key tiles K_j, V_j through a shared-memory ring.  Warp roles:
+//   warps 0-3   softmax for Q0 (one query row per thread, TMEM lanes 0-127)
+//   warps 4-7   softmax for Q1
+//   warp  8     tcgen05 MMA issue (one thread)
+//   warp  9     TMA producer (one thread)
+// Tensor memory (512 columns): S_t = Q_t K_j^T (fp32, 128 columns) at
+// column 128 t; P_t (bf16, 64 columns) overwrites the first half of S_t and is
+// the A operand of O_t += P_t V_j; O_t (fp32, D columns) at 256 + D t.
+// The two Q tiles ping-pong: while one tile's softmax runs, the tensor core
+// works on the other tile's MMAs.
+//
+// Online softmax in base 2: x = s * scale * log2(e); m is a running row
+// maximum that is only raised (and O, l rescaled) when the tile maximum
+// exceeds it by more than 8, i.e. a factor 256.  Every P and l use the same
+// stale m, so the final O / l is exact; P values stay below 256.
+#pragma once
+
+#include "dropout_hash.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdArgs {
+  int B, H, N;
+  float scale_log2;         // scale * log2(e)
+  uint32_t drop_threshold;  // keep iff hash32 >= threshold
+  float drop_scale;         // 1 / (1 - p)
+  uint64_t seed;
+  __nv_bfloat16* o;  // [B,H,N,D]
+  float* lse;        // [B,H,N], natural log
+  int* err;          // device error word (may be null)
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kHalf = 128u * 128u;     // one 128-row x 64-column bf16 half tile
+  static constexpr uint32_t kTile = 128u * D * 2u;   // one 128 x D bf16 tile
+  static constexpr int kStages = D == 128 ? 4 : 8;   // K/V ring depth
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = kOffQ + 2 * kTile;
+  static constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  static constexpr uint32_t kColO = 256;  // O_t at kColO + D * t
+};
+
+template <int D, bool CAUSAL, bool DROPOUT>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  using L = FwdLayout<D>;
+  static_assert(D == 64 || D == 128, "head dim");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* bar_q = bars;                               // [2]   Q_t landed
+  uint64_t* bar_kv_full = bars + 2;                     // [S]   K/V stage landed
+  uint64_t* bar_kv_empty = bar_kv_full + L::kStages;    // [S]   K/V stage consumed
+  uint64_t* bar_s = bar_kv_empty + L::kStages;          // [2]   S_t ready in TMEM
+  uint64_t* bar_p = bar_s + 2;                          // [2]   P_t written (128 arrivals)
+  uint64_t* bar_pv = bar_p + 2;                         // [2]   O_t += P_t V_j done
+  uint64_t* bar_drain = bar_pv + 2;                     //       all MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  const uint32_t sbase = smem_u32(smem);
+
+  // Work tile.  For the causal mask the CTA with the most key tiles goes
+  // first (longest-processing-time order across the grid).
+  const int BH = a.B * a.H;
+  const int n_cta_tiles = (a.N + 255) >> 8;
+  const int tile_rev = blockIdx.x / BH;
+  const int bh = blockIdx.x - tile_rev * BH;
+  const int cta_tile = CAUSAL ? (n_cta_tiles - 1 - tile_rev) : tile_rev;
+  const int n_kv_all = (a.N + 127) >> 7;
+  const int qt0 = 2 * cta_tile;
+  const bool act1 = (qt0 + 1) * 128 < a.N;
+  const int nkv0 = CAUSAL ? qt0 + 1 : n_kv_all;
+  const int nkv1 = act1 ? (CAUSAL ? qt0 + 2 : n_kv_all) : 0;
+  const int nkv_max = nkv0 > nkv1 ? nkv0 : nkv1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q[0], 1);
+    mbar_init(&bar_q[1], 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&bar_kv_full[s], 1);
+      mbar_init(&bar_kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s[t], 1);
+      mbar_init(&bar_p[t], 128);
+      mbar_init(&bar_pv[t], 1);
+    }
+    mbar_init(bar_drain, 1);
+    const bool misaligned = (sbase & 1023u) != 0u;
+    *abort_flag = misaligned ? 1 : 0;
+    if (misaligned && a.err) atomicCAS(a.err, kDevOk, kDevMisaligned);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, a.err};
+  const bool run = *abort_flag == 0;
+
+  if (run && warp == 9) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const uint64_t pol_keep = policy_evict_last();   // K/V: re-read by every Q tile of the head
+      const uint64_t pol_once = policy_evict_first();  // Q: read once
+      for (int t = 0; t < 2; ++t) {
+        if (t == 1 && !act1) break;
+        mbar_arrive_expect_tx(&bar_q[t], L::kTile);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, (qt0 + t) * 128, bh,
+                      &bar_q[t], pol_once);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv_max && ok; ++j) {
+        for (int which = 0; which < 2; ++which) {
+          if (!mbar_wait(&bar_kv_empty[stage], phase ^ 1u, ab)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
+          const CUtensorMap* m = which ? &tm_v : &tm_k;
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, j * 128, bh,
+                        &bar_kv_full[stage], pol_keep);
+          ++issued;
+          if (++stage == L::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Every load issued must land before the CTA may exit.
+      mbar_wait_drain(&bar_q[0], 0);
+      if (act1) mbar_wait_drain(&bar_q[1], 0);
+      const int first = issued > L::kStages ? issued - L::kStages : 0;
+      for (int n = first; n < issued; ++n) mbar_wait_drain(&bar_kv_full[n % L::kStages], (n / L::kStages) & 1);
+    }
+  } else if (run && warp == 8) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // S = Q K^T, both K-major
+      constexpr uint32_t kIdO = idesc_bf16(128, D, false, true);     // O += P V, V is MN-major
+      bool ok = mbar_wait(&bar_q[0], 0, ab) && (!act1 || mbar_wait(&bar_q[1], 0, ab));
+      tc_fence_after();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued_any = false;
+      for (int j = 0; j < nkv_max && ok; ++j) {
+        // S_t = Q_t K_j^T
+        if (!mbar_wait(&bar_kv_full[stage], phase, ab)) break;
+        tc_fence_after();
+        const uint32_t sK = sbase + L::kOffKV + stage * L::kTile;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= (t ? nkv1 : nkv0)) continue;
+          // S_t shares its columns with P_t, which O_t += P_t V_{j-1} reads.
+          if (j > 0) {
+            if (!mbar_wait(&bar_pv[t], (j - 1) & 1, ab)) {
+              ok = false;
+              continue;
+            }
+            tc_fence_after();
+          }
+          const uint32_t sQ = sbase + L::kOffQ + t * L::kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + 128u * t, desc_kmajor(sQ, kk, L::kHalf), desc_kmajor(sK, kk, L::kHalf), kIdS,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(&bar_s[t]);
+          issued_any = true;
+        }
+        if (!ok) break;
+        mma_commit(&bar_kv_empty[stage]);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        // O_t += P_t V_j
+        if (!mbar_wait(&bar_kv_full[stage], phase, ab)) break;
+        tc_fence_after();
+        const uint32_t sV = sbase + L::kOffKV + stage * L::kTile;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= (t ? nkv1 : nkv0)) continue;
+          if (!mbar_wait(&bar_p[t], j & 1, ab)) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar_pv[t]);
+        }
+        if (!ok) break;
+        mma_commit(&bar_kv_empty[stage]);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (issued_any) {
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else if (run && warp < 8) {
+    // ---------------------------------------------------------- softmax
+    const int t = warp >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // row within the Q tile == TMEM lane
+    if (t == 0 || act1) {
+      const int nkv = t ? nkv1 : nkv0;
+      const int q_row = (qt0 + t) * 128 + r;
+      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+      const uint32_t tS = tmem + lane_off + 128u * t;
+      const uint32_t tO = tmem + lane_off + L::kColO + D * t;
+      const float sl2 = a.scale_log2;
+      float m_used = -INFINITY;  // running maximum (base-2 units) the P values are taken against
+      float l = 0.f;             // running sum of undropped P
+      uint32_t rkey = 0;
+      if (DROPOUT) rkey = dropout_row_key(a.seed, (uint32_t)(bh / a.H), (uint32_t)(bh % a.H), (uint32_t)q_row);
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait(&bar_s[t], j & 1, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t u[4][32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
+        const bool last = j == nkv - 1;
+        // key 128 j + c is visible to query 128 (qt0 + t) + r iff c < lim
+        int lim = 128;
+        if (CAUSAL && last) lim = r + 1;                          // diagonal tile
+        if (!CAUSAL && last && (a.N & 127)) lim = a.N - j * 128;  // padded keys past N
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < lim) mx = fmaxf(mx, __uint_as_float(u[c >> 5][c & 31]));
+        const float m_new = fmaxf(m_used, mx * sl2);
+        if (__any_sync(0xffffffffu, m_new > m_used + 8.0f)) {
+          const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
+          l *= alpha;
+          m_used = m_new;
+          if (j > 0) {
+            // O_t holds the sum over earlier tiles; O_t += P V_{j-1} has
+            // retired (it completed before S_t(j) was issued).  The score
+            // registers are released for the rescale and reloaded after it.
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+              uint32_t o[32];
+              tmem_ld32_sync(tO + 32u * c4, o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(tO + 32u * c4, o);
+            }
+            tmem_st_wait();
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
+          }
+        }
+        const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+        float psum = 0.f;
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x0 = 2 * c < lim ? __uint_as_float(u[(2 * c) >> 5][(2 * c) & 31]) : -INFINITY;
+          const float x1 = 2 * c + 1 < lim ? __uint_as_float(u[(2 * c + 1) >> 5][(2 * c + 1) & 31]) : -INFINITY;
+          float p0 = ex2(fmaf(x0, sl2, -msub));
+          float p1 = ex2(fmaf(x1, sl2, -msub));
+          psum += p0 + p1;
+          if (DROPOUT) {
+            const uint32_t col = (uint32_t)(j * 128 + 2 * c);
+            p0 = dropout_hash(rkey, col) >= a.drop_threshold ? p0 * a.drop_scale : 0.f;
+            p1 = dropout_hash(rkey, col + 1) >= a.drop_threshold ? p1 * a.drop_scale : 0.f;
+          }
+          pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
+        }
+        l += psum;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) tmem_st16(tS + 16u * c16, pk[c16]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_p[t]);
+      }
+      // epilogue: O = O_t / l, lse = (m + log2 l) ln 2
+      if (ok && mbar_wait(&bar_pv[t], (nkv - 1) & 1, ab)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool in_range = q_row < a.N;
+        __nv_bfloat16* orow = a.o + ((size_t)bh * a.N + (size_t)(in_range ? q_row : 0)) * D;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t o[32];
+          tmem_ld32_sync(tO + 32u * c4, o);
+          uint32_t w[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            w[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+          if (in_range) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_global_v4(orow + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
+        }
+        if (in_range) a.lse[(size_t)bh * a.N + q_row] = (m_used + log2f(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,107 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every symbol ``include/fa.h`` declares, and
+reject invalid arguments with the documented status codes before touching
+the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from io_aware_exact_25_b200 import binding
+from io_aware_exact_25_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "fa_fwd" in names and "fa_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(binding.EXPORTS) == set(names)
+
+
+def test_status_codes_match_header(lib):
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    codes = dict((k, int(v)) for k, v in re.findall(r"(FA_[A-Z_]+)\s*=\s*(-?\d+)", text))
+    for k, v in codes.items():
+        assert getattr(binding, k) == v
+        assert lib.fa_strerror(v) and lib.fa_strerror(v).decode() != "unknown status"
+    assert lib.fa_strerror(12345).decode() == "unknown status"
+    assert lib.fa_version() == 100
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=128, d=64, scale=0.125, causal=0, p=0.0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, p, 0, None)
+
+
+def _bwd(lib, ptr=16, lse=16, B=1, H=1, N=128, d=64, scale=0.125, causal=0, p=0.0, ws=16, wsb=1 << 30):
+    return lib.fa_bwd(ptr, ptr, ptr, ptr, ptr, lse, ptr, ptr, ptr, B, H, N, d, scale, causal, p, 0, ws, wsb,
+                      None)
+
+
+def test_invalid_arguments_are_rejected_before_launch(lib):
+    assert _fwd(lib, d=96) == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, B=-1) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, N=-5) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf")) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, causal=2) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, p=1.0) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, p=-0.1) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, q=None) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, lse=None) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, q=24) == binding.FA_ERR_ALIGNMENT      # 8-byte aligned only
+    assert _fwd(lib, o=18) == binding.FA_ERR_ALIGNMENT
+    assert _fwd(lib, lse=18) == binding.FA_ERR_ALIGNMENT
+    assert _fwd(lib, B=1 << 25) == binding.FA_ERR_TOO_LARGE
+    assert _bwd(lib, ws=None) == binding.FA_ERR_WORKSPACE
+    assert _bwd(lib, wsb=100) == binding.FA_ERR_WORKSPACE
+    assert _bwd(lib, ws=24) == binding.FA_ERR_ALIGNMENT
+    assert _bwd(lib, ptr=None) == binding.FA_ERR_INVALID_ARG
+    assert _bwd(lib, d=80) == binding.FA_ERR_UNSUPPORTED
+    assert _bwd(lib, p=1.5) == binding.FA_ERR_INVALID_ARG
+
+
+def test_empty_problems_are_noops(lib):
+    # nothing to do: success without touching the (absent) device or pointers
+    assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == binding.FA_OK
+    assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == binding.FA_OK
+    assert _bwd(lib, ptr=None, lse=None, H=0, ws=None, wsb=0) == binding.FA_OK
+    assert lib.fa_dropout_mask(1, 1, 0, 0.1, 0, None, 0, None, 0, None, None) == binding.FA_OK
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 128, 64), (2, 16, 8192, 128), (1, 3, 300, 128), (1, 1, 1, 64)])
+def test_workspace_size_formula(lib, B, H, N, d):
+    npad = (N + 127) // 128 * 128
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    expect = up(B * H * N * d * 4) + 2 * up(B * H * npad * 4)
+    assert lib.fa_bwd_workspace_size(B, H, N, d) == expect
+    assert lib.fa_bwd_workspace_size(B, H, N, 96) == 0
+    assert lib.fa_bwd_workspace_size(0, H, N, d) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.fwd(x, x, x)

@@ -1,0 +1,206 @@
+"""GPU parity: the sm_100a kernels (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 inputs and outputs, fp32 accumulation): for O, dQ, dK, dV
+max |err| <= 2e-2 and relative L2 error <= 5e-3; lse within 1e-3; dropout
+keep masks bit-exact.  Small cases compare every element; the long-context
+workloads compare sampled query rows (O, lse, dQ) and sampled key rows
+(dK, dV) the oracle computes one by one, plus identities that hold at any
+size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_25_b200 import binding
+from io_aware_exact_25_b200.inputs import WORKLOADS, make_inputs, sample_rows, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+LSE_ABS = 1e-3
+
+
+def _check(name, got, ref):
+    g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    assert np.all(np.isfinite(g)), f"{name}: non-finite output"
+    err = np.abs(g - ref)
+    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= MAX_ABS, f"{name}: max abs err {err.max():.3e}"
+    assert rel <= REL_L2, f"{name}: rel L2 err {rel:.3e}"
+
+
+def _check_lse(got, ref):
+    g = got.detach().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    err = np.abs(g - ref).max()
+    assert err <= LSE_ABS, f"lse: max abs err {err:.3e}"
+
+
+def _to(x, dev):
+    return {n: t.to(dev) for n, t in x.items()}
+
+
+def _run(xd, causal, scale, p=0.0, seed=0, backward=True):
+    o, lse = binding.fwd(xd["q"], xd["k"], xd["v"], causal=causal, scale=scale, dropout_p=p, seed=seed)
+    grads = None
+    if backward:
+        grads = binding.bwd(xd["q"], xd["k"], xd["v"], o, xd["do"], lse, causal=causal, scale=scale,
+                            dropout_p=p, seed=seed)
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    return o, lse, grads
+
+
+def _full_compare(x, o, lse, grads, scale, causal, p=0.0, seed=0):
+    B, H, N, d = x["q"].shape
+    ro, rlse = oracle.forward(x["q"], x["k"], x["v"], scale, causal=causal, p_drop=p, seed=seed)
+    _check("O", o, ro)
+    _check_lse(lse, rlse)
+    if grads is not None:
+        dq, dk, dv = grads
+        rdq, _, dev = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], scale, causal=causal, p_drop=p, seed=seed)
+        rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], scale, causal=causal, p_drop=p, seed=seed)
+        assert dev < 1e-9
+        _check("dQ", dq, rdq)
+        _check("dK", dk, rdk)
+        _check("dV", dv, rdv)
+
+
+# ------------------------------------------------------------ small cases
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_workload_all_elements(cuda_device, causal):
+    w = WORKLOADS["tiny"]
+    x = workload_inputs(w)
+    o, lse, grads = _run(_to(x, cuda_device), causal, w.scale)
+    _full_compare(x, o, lse, grads, w.scale, causal)
+
+
+@pytest.mark.parametrize("N,d", [(1, 64), (77, 128), (129, 64), (300, 128), (640, 64), (1000, 128)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ragged_and_multi_tile_lengths(cuda_device, N, d, causal):
+    """Lengths that are not a multiple of the 128-row tile, below one tile,
+    and spanning several tiles with a ragged tail."""
+    x = make_inputs(2, 3, N, d, seed=N + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse, grads = _run(_to(x, cuda_device), causal, scale)
+    _full_compare(x, o, lse, grads, scale, causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_non_default_scale_and_peaked_rows(cuda_device, d):
+    x = make_inputs(1, 4, 512, d, seed=21, offset_norm=2.0)
+    scale = 0.7 / math.sqrt(d)
+    for causal in (False, True):
+        o, lse, grads = _run(_to(x, cuda_device), causal, scale)
+        _full_compare(x, o, lse, grads, scale, causal)
+
+
+def test_large_score_range_triggers_rescaling(cuda_device):
+    """Row maxima that grow across key tiles exercise the online rescaling
+    of O and l (scores spanning hundreds in base-2 units)."""
+    g = torch.Generator().manual_seed(5)
+    B, H, N, d = 1, 2, 768, 64
+    q = torch.randn(B, H, N, d, generator=g)
+    k = torch.randn(B, H, N, d, generator=g) * torch.linspace(0.2, 6.0, N).view(1, 1, N, 1)
+    v = torch.randn(B, H, N, d, generator=g)
+    do = torch.randn(B, H, N, d, generator=g)
+    x = {n: t.to(torch.bfloat16).contiguous() for n, t in zip(("q", "k", "v", "do"), (q, k, v, do))}
+    for causal in (False, True):
+        o, lse, grads = _run(_to(x, cuda_device), causal, 1.0 / math.sqrt(d))
+        _full_compare(x, o, lse, grads, 1.0 / math.sqrt(d), causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_small_all_elements(cuda_device, d, causal):
+    p, seed = 0.1, 4
+    x = make_inputs(1, 2, 384, d, seed=31)
+    scale = 1.0 / math.sqrt(d)
+    o, lse, grads = _run(_to(x, cuda_device), causal, scale, p=p, seed=seed)
+    _full_compare(x, o, lse, grads, scale, causal, p=p, seed=seed)
+
+
+def test_dropout_mask_bit_exact(cuda_device):
+    B, H, N = 2, 3, 1000
+    heads = [0, 4, 5]
+    rows = [0, 1, 17, 500, 999]
+    for p, seed in ((0.1, 4), (0.5, 2 ** 40 + 7), (0.0, 1)):
+        got = binding.dropout_mask(B, H, N, p, seed, heads, rows, device=cuda_device).cpu().numpy()
+        ref = oracle.dropout_mask(B, H, N, p, seed, heads=heads, rows=rows)
+        assert np.array_equal(got, ref)
+
+
+def test_empty_problem_is_noop(cuda_device):
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.bfloat16, device=cuda_device)
+    o, lse = binding.fwd(q, q, q, causal=True)
+    assert o.shape == q.shape and lse.shape == (1, 2, 0)
+
+
+@pytest.mark.parametrize("name", ["train2k", "train2k_causal"])
+def test_training_shape_all_rows(cuda_device, name):
+    w = WORKLOADS[name]
+    x = workload_inputs(w)
+    o, lse, grads = _run(_to(x, cuda_device), w.causal, w.scale)
+    _full_compare(x, o, lse, grads, w.scale, w.causal)
+
+
+# ------------------------------------------------- long-context workloads
+
+def _sampled_compare(w, n_rows, kv_heads, kv_keys):
+    x = workload_inputs(w)
+    xd = _to(x, "cuda")
+    o, lse, grads = _run(xd, w.causal, w.scale, p=w.p_drop, seed=w.seed)
+    dq, dk, dv = grads
+    BH = w.B * w.H
+    rows = sample_rows(w.N, n_rows, w.seed)
+    ro, rlse = oracle.forward(x["q"], x["k"], x["v"], w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed,
+                              rows=rows)
+    ridx = torch.as_tensor(rows, device="cuda")
+    _check("O rows", o.view(BH, w.N, w.d)[:, ridx], ro)
+    _check_lse(lse.view(BH, w.N)[:, ridx], rlse)
+    rdq, _, dev = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], w.scale, causal=w.causal, p_drop=w.p_drop,
+                                    seed=w.seed, rows=rows)
+    assert dev < 1e-9
+    _check("dQ rows", dq.view(BH, w.N, w.d)[:, ridx], rdq)
+    rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], w.scale, causal=w.causal, p_drop=w.p_drop,
+                                  seed=w.seed, heads=kv_heads, keys=kv_keys)
+    hidx = torch.as_tensor(kv_heads, device="cuda")
+    kidx = torch.as_tensor(kv_keys, device="cuda")
+    _check("dK rows", dk.view(BH, w.N, w.d)[hidx][:, kidx], rdk)
+    _check("dV rows", dv.view(BH, w.N, w.d)[hidx][:, kidx], rdv)
+    # identities over every head and key (any size): sum_j dK_j = 0 and, without
+    # dropout, sum_j dV_j = sum_i dO_i; both in fp32 sums of bf16 outputs
+    sdk = dk.float().sum(dim=2)
+    scale_dk = dk.float().abs().sum(dim=2)
+    assert (sdk.abs() <= 1e-2 * scale_dk + 1e-2).all()
+    if w.p_drop == 0.0:
+        sdv = dv.float().sum(dim=2)
+        sdo = xd["do"].float().sum(dim=2)
+        assert ((sdv - sdo).abs() <= 1e-2 * dv.float().abs().sum(dim=2) + 1e-2).all()
+    if w.p_drop > 0.0:
+        mrows = rows[:16]
+        got = binding.dropout_mask(w.B, w.H, w.N, w.p_drop, w.seed, list(range(BH)), mrows).cpu().numpy()
+        ref = oracle.dropout_mask(w.B, w.H, w.N, w.p_drop, w.seed, rows=mrows)
+        assert np.array_equal(got, ref)
+
+
+def test_long8k_causal_sampled(cuda_device):
+    w = WORKLOADS["long8k_causal"]
+    keys = sample_rows(w.N, 64, w.seed + 100)
+    _sampled_compare(w, 512, kv_heads=[0, w.B * w.H - 1], kv_keys=keys)
+
+
+def test_long32k_causal_sampled(cuda_device):
+    w = WORKLOADS["long32k_causal"]
+    keys = sorted(set([w.N - 1, w.N - 128, w.N - 1500] + list(range(w.N - 2048, w.N, 97))))
+    _sampled_compare(w, 256, kv_heads=[0, w.H - 1], kv_keys=keys)
+
+
+def test_long64k_causal_dropout_sampled(cuda_device):
+    w = WORKLOADS["long64k_causal_dropout"]
+    keys = sorted(set([w.N - 1, w.N - 200] + list(range(w.N - 1024, w.N, 61))))
+    _sampled_compare(w, 128, kv_heads=[3], kv_keys=keys)
