@@ -1,0 +1,425 @@
+#!/usr/bin/env python3
+"""Benchmark: causal bf16 attention forward + backward through the C ABI.
+
+One step = one pass of the whole path over one batch: fa_fwd (fused tiled
+forward, online softmax, lse) then the backward (row pass, fused recompute
+kernel, dQ conversion).  Default workload: B=2, H=16, N=8192, d=128, causal,
+no dropout -- the long-context configuration the TFLOPS target is stated for
+(N >= 8192, d = 128).  FLOPs follow the attention convention:
+4*B*H*N^2*d forward, halved when causal, and 2.5x that backward.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (its own
+B*H heads; heads are independent, so there is no collective on the data
+path) and the job's value is the total FLOPs of all ranks over the slowest
+rank's time ("weak" scaling).
+
+``--impl reference`` times the fp64 CPU oracle (the only other
+implementation of this path) on the host cores instead, on a bounded sample
+of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd and fwd+bwd TFLOPS (bf16, causal) and % of B200 BF16 tensor peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------- traffic record
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("bwd_sm100.cuh", "fwd_sm100.cuh", "sm100.cuh", "dropout_hash.cuh", "fa_api.cu"):
+        with open(os.path.join(ROOT, "io_aware_exact_25_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# ------------------------------------------------------- oracle (CPU)
+
+def oracle_step(x, w, n_rows: int):
+    """fp64 oracle forward + full backward on the causal prefix of length
+    n_rows of head (b=0, h=0): an exact sub-problem of the workload (causal
+    rows < n_rows see only keys < n_rows).  Returns (seconds, FLOPs)."""
+    import oracle
+    q, k, v, do = (x[n][:1, :1, :n_rows].contiguous() for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    oracle.backward_q(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    oracle.backward_kv(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    dt = time.perf_counter() - t0
+    f = 4.0 * n_rows * n_rows * w.d / (2.0 if w.causal else 1.0)
+    return dt, 3.5 * f
+
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from io_aware_exact_25_b200.inputs import workload_inputs
+    import oracle
+    x = workload_inputs(w)
+    n_rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_step(x, w, n_rows)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, f = oracle_step(x, w, n_rows)
+        tot_t += dt
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"per step: fwd+bwd of the causal prefix N={n_rows} of head (0,0)"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
+                        f"{'causal' if w.causal else 'non-causal'} dropout={w.p_drop} bf16",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "dropout_p": w.p_drop,
+            "l2": "inputs larger than L2 (Q, K, V, dO: 4 x 64 MiB per step > 126 MB L2)",
+            "parallelism": "replicas: each GPU runs its own B*H heads, no collective"}
+
+
+# ------------------------------------------------------------ our arm
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from io_aware_exact_25_b200 import binding
+    from io_aware_exact_25_b200.inputs import workload_inputs
+    lib = binding.load()
+
+    x = workload_inputs(w)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = binding.bwd_workspace_size(B, H, N, d)
+    work = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    causal = int(w.causal)
+    P = binding._ptr
+
+    def check(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: {binding.strerror(rc)}")
+
+    def fwd():
+        check(lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, w.scale, causal, w.p_drop, w.seed, s),
+              "fa_fwd")
+
+    def bwd_prepare():
+        check(lib.fa_bwd_prepare(P(o), P(do), P(lse), B, H, N, d, P(work), wsb, s), "fa_bwd_prepare")
+
+    def bwd_recompute():
+        check(lib.fa_bwd_recompute(P(q), P(k), P(v), P(do), P(dk), P(dv), B, H, N, d, w.scale, causal,
+                                   w.p_drop, w.seed, P(work), wsb, s), "fa_bwd_recompute")
+
+    def bwd_finalize():
+        check(lib.fa_bwd_finalize(P(dq), B, H, N, d, w.scale, P(work), wsb, s), "fa_bwd_finalize")
+
+    stages = [("fwd_kernel", fwd), ("bwd_pre_kernel", bwd_prepare), ("bwd_kernel", bwd_recompute),
+              ("bwd_post_kernel", bwd_finalize)]
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        for _, fn in stages:
+            fn()
+    torch.cuda.synchronize(dev)
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error during warm-up")
+
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    time.sleep(0.3)
+
+    # device-timed region: events between the stage launches on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for st in range(args.steps):
+        ev[st][0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            ev[st][i + 1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_stage_ms = [sum(ev[st][i].elapsed_time(ev[st][i + 1]) for st in range(args.steps)) / args.steps
+                    for i in range(len(stages))]
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error in the timed region")
+
+    if args.no_extras:
+        if rank == 0:
+            print(json.dumps({"profiling_run": True, "ms_per_step": elapsed_ms / args.steps,
+                              "stage_ms": dict(zip([n for n, _ in stages], per_stage_ms))}), flush=True)
+        if ws > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # end to end: pinned host inputs -> device, fwd + bwd, results -> pinned host
+    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
+    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+    hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hlse))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        do.copy_(hdo, non_blocking=True)
+        binding.fwd(q, k, v, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed, o=o, lse=lse)
+        binding.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
+                    dq=dq, dk=dk, dv=dv, workspace=work)
+        ho.copy_(o, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+
+    # max over ranks
+    times = torch.tensor([elapsed_ms, e2e_ms] + per_stage_ms, dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(times[0]), float(times[1])
+    per_stage_ms = [float(t) for t in times[2:]]
+
+    if rank == 0:
+        ff, fb = w.fwd_flops(), w.bwd_flops()
+        ms_step = elapsed_ms / args.steps
+        value = ws * (ff + fb) / (ms_step * 1e-3) / 1e12
+        fwd_ms = per_stage_ms[0]
+        bwd_ms = sum(per_stage_ms[1:])
+        peaks, peak_kind = load_peaks()
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        # dominant kernel: the largest share of the step
+        names = [n for n, _ in stages]
+        dom = max(range(len(stages)), key=lambda i: per_stage_ms[i])
+        dom_flops = {0: ff, 2: fb}.get(dom)
+        if dom_flops is not None:
+            achieved = dom_flops / (per_stage_ms[dom] * 1e-3) / 1e12
+            roof = {"bound": "tensor", "kernel": names[dom], "achieved": achieved, "peak": sustained,
+                    "unit": "TFLOP/s", "frac": achieved / sustained,
+                    "peak_note": f"bf16_tflops_sustained of {peak_kind} (kernel timed inside a long step loop)",
+                    "frac_of_burst": achieved / burst, "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,
+                    "traffic": recorded_traffic(names[dom], w.name),
+                    "algorithmic_flops_per_launch": dom_flops}
+        else:
+            roof = {"bound": "hbm", "kernel": names[dom], "achieved": None, "peak": None, "unit": "GB/s",
+                    "frac": None, "traffic": None}
+        # oracle baseline on the host cores (bounded sample of the same workload)
+        import oracle
+        cpu_dt, cpu_f = oracle_step(x, w, args.cpu_rows)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w),
+            "fwd_tflops": ws * ff / (fwd_ms * 1e-3) / 1e12,
+            "fwd_bwd_tflops": value,
+            "frac_of_peak": {
+                "fwd_vs_burst": (ff / (fwd_ms * 1e-3) / 1e12) / burst,
+                "fwd_bwd_vs_burst": (value / ws) / burst,
+                "fwd_vs_datasheet": (ff / (fwd_ms * 1e-3) / 1e12) / DATASHEET_BF16_TFLOPS,
+                "fwd_bwd_vs_datasheet": (value / ws) / DATASHEET_BF16_TFLOPS,
+                "peaks": f"{peak_kind}: burst {burst}, sustained {sustained}, datasheet {DATASHEET_BF16_TFLOPS}"},
+            "stage_ms": dict(zip(names, per_stage_ms)),
+            "roofline": roof,
+            "cpu_baseline": {"value": cpu_f / cpu_dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"fp64 fwd+bwd of the causal prefix N={args.cpu_rows} of head (0,0) "
+                                       f"({cpu_dt:.1f} s)"},
+            "e2e": {"value": ws * (ff + fb) * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "binding.fwd/binding.bwd (C ABI) with pinned host buffers"},
+            "gpu_launches": args.steps * len(stages),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long8k_causal")
+    ap.add_argument("--cpu-rows", type=int, default=8192,
+                    help="causal prefix length of the oracle baseline sample")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the end-to-end and CPU-baseline legs (profiling runs)")
+    ap.add_argument("--ref-rows", type=int, default=1024,
+                    help="causal prefix length per step of the reference (oracle) arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from io_aware_exact_25_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

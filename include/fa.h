@@ -96,6 +96,26 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            uint64_t seed, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The three stages fa_bwd runs, callable one by one on the same stream (for
+ * overlap with other work or per-stage timing).  Same arguments and checks as
+ * fa_bwd; running them in order is exactly fa_bwd.
+ *   fa_bwd_prepare:   D_i = dO_i . O_i ("FlashAttention for Efficient
+ *                     Training" section 3.2: the chain rule through the
+ *                     row-wise softmax needs this row dot), lse in base 2,
+ *                     and a zeroed fp32 dQ accumulator, all in workspace.
+ *   fa_bwd_recompute: the fused recompute kernel; writes dk, dv and adds
+ *                     the dQ partials into the workspace accumulator.
+ *   fa_bwd_finalize:  dq = scale * accumulator, rounded to bf16.
+ */
+int fa_bwd_prepare(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
+                   void* workspace, size_t workspace_bytes, void* stream);
+int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
+                     int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                     void* workspace, size_t workspace_bytes, void* stream);
+int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
  * Debug export of the dropout mask: for each listed head bh = b*H + h
  * (heads[nheads]) and query row (rows[nrows]), writes the keep bit of every
  * key j < N to out[(hi * nrows + ri) * N + j] (1 = kept).  heads, rows and

@@ -27,8 +27,9 @@ FA_ERR_CUDA = -5
 FA_ERR_DEVICE = -6
 FA_ERR_TOO_LARGE = -7
 
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_dropout_mask", "fa_strerror",
-           "fa_last_cuda_error", "fa_get_device_error", "fa_version")
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
+           "fa_bwd_finalize", "fa_dropout_mask", "fa_strerror", "fa_last_cuda_error",
+           "fa_get_device_error", "fa_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -55,11 +56,15 @@ def load() -> ctypes.CDLL:
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
+        lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
+        lib.fa_bwd_recompute.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
+        lib.fa_bwd_finalize.argtypes = [vp, I, I, I, I, F, vp, SZ, vp]
         lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
-        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_dropout_mask, lib.fa_get_device_error,
+        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
+                   lib.fa_bwd_finalize, lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
         _lib = lib
@@ -135,6 +140,32 @@ def bwd(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, 
                        _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                        _stream(stream))
     _call(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_stages(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, dq=None,
+               dk=None, dv=None, workspace=None, stream=None):
+    """The backward as its three C-ABI stages (prepare, recompute, finalize)."""
+    _check_inputs(q, k, v, o, dout)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    wsb = int(workspace.numel() * workspace.element_size())
+    s = _stream(stream)
+    lib = load()
+    _call(lib.fa_bwd_prepare(_ptr(o), _ptr(dout), _ptr(lse), B, H, N, d, _ptr(workspace), wsb, s),
+          "fa_bwd_prepare")
+    _call(lib.fa_bwd_recompute(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d,
+                               float(scale), int(bool(causal)), float(dropout_p), int(seed),
+                               _ptr(workspace), wsb, s), "fa_bwd_recompute")
+    _call(lib.fa_bwd_finalize(_ptr(dq), B, H, N, d, float(scale), _ptr(workspace), wsb, s),
+          "fa_bwd_finalize")
     return dq, dk, dv
 
 

@@ -154,11 +154,17 @@ struct BwdLayout {
   static constexpr uint32_t kOffDS = kOffDO + kDoStages * kTile;  // dS, 128 x 128 bf16, MN-major halves
   static constexpr uint32_t kRowStage = 3u * 128u * 4u;             // lse2, D, dropout row keys
   static constexpr uint32_t kOffRow = kOffDS + 2u * kHalf;
-  static constexpr uint32_t kOffBar = kOffRow + 2u * kRowStage;
+  // dQ staging: three 128-row x 16-column fp32 pieces (64-byte rows,
+  // 64-byte swizzle), the source tiles of the TMA reductions
+  static constexpr uint32_t kDqPiece = 128u * 64u;
+  static constexpr int kDqBufs = 3;
+  static constexpr uint32_t kOffDQ = kOffRow + 2u * kRowStage;
+  static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
   // row_empty[2], s, dp, p, ds, dv, dk, dq, dq_free, drain
   static constexpr int kNumBars = 1 + 12 + 9;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  static_assert(kOffDQ % 1024 == 0, "staging tiles must be swizzle-aligned");
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
@@ -170,7 +176,7 @@ template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdArgs a) {
+               const __grid_constant__ CUtensorMap tm_dqacc, const BwdArgs a) {
   using L = BwdLayout<D>;
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -195,12 +201,16 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* bar_dq_free = bars + 20;
   uint64_t* bar_drain = bars + 21;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);  // [0] abort, [1] dQ warpgroup flag
   const uint32_t sbase = smem_u32(smem);
 
   const int BH = a.B * a.H;
   const int nT = (a.N + 127) >> 7;
-  const int jt = blockIdx.x / BH;  // key tile; ascending = most query tiles first when causal
+  // CTA order: key tiles ascending (the most query tiles first when causal:
+  // longest-processing-time order), heads interleaved.  The CTAs of a wave
+  // sweep the query tiles of their heads in near lockstep, so the Q/dO tiles
+  // and accumulator rows they share stay in L2.
+  const int jt = blockIdx.x / BH;  // key tile
   const int bh = blockIdx.x - jt * BH;
   const int i_begin = CAUSAL ? jt : 0;
   const int n_steps = nT - i_begin;
@@ -249,6 +259,7 @@ __global__ void __launch_bounds__(448, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_dqacc);
       mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
       for (int h = 0; h < D / 64; ++h) {
         tma_load_3d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, bh, bar_kv, pol_keep);
@@ -388,14 +399,26 @@ __global__ void __launch_bounds__(448, 1)
     }
   } else if (run && warp >= 8 && warp < 12) {
     // ------------------------------------------ dQ read-out + accumulate
+    // The partial dQ_i (128 rows x D fp32, query rows on the TMEM lanes) is
+    // added into the fp32 accumulator in 16-column pieces: every thread
+    // writes its row of the piece into a 64-byte-swizzled staging tile, and
+    // one thread issues a tiled TMA reduction of the whole 128 x 16 tile.
+    // Three staging tiles rotate; a tile is rewritten only after the
+    // reduction issued from it three pieces earlier has read it.  The loop is
+    // uniform over the warpgroup (one thread waits, a named barrier shares
+    // the outcome), so every thread reaches every named barrier.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query within the tile == TMEM lane
+    const bool leader = warp == 8 && lane == 0;
     const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDP;
+    volatile int* dq_flag = abort_flag + 1;
+    uint32_t piece = 0;
     for (int it = 0; it < n_steps; ++it) {
-      if (!mbar_wait(bar_dq, it & 1, ab)) break;
+      if (leader) *dq_flag = mbar_wait(bar_dq, it & 1, ab) ? 1 : 0;
+      named_bar_sync(1, 128);
+      if (*dq_flag == 0) break;
       tc_fence_after();
-      const int q_row = (i_begin + it) * 128 + row;
-      float* dst = a.dq_acc + ((size_t)bh * a.N + (size_t)(q_row < a.N ? q_row : 0)) * D;
+      const int q0 = (i_begin + it) * 128;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t v[32];
@@ -404,14 +427,27 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_before();
           mbar_arrive(bar_dq_free);
         }
-        if (q_row < a.N) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            red_add_v4(dst + 32 * c4 + 4 * k, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+        for (int h = 0; h < 2; ++h, ++piece) {
+          const uint32_t buf = sbase + L::kOffDQ + (piece % L::kDqBufs) * L::kDqPiece;
+          const uint32_t rbase = buf + (uint32_t)row * 64u;
+          const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            st_shared_v4(rbase + (((uint32_t)q4 ^ sw) << 4), v[16 * h + 4 * q4], v[16 * h + 4 * q4 + 1],
+                         v[16 * h + 4 * q4 + 2], v[16 * h + 4 * q4 + 3]);
+          fence_proxy_async_smem();
+          // the tile the next piece writes was last read by piece - 2
+          if (leader) bulk_wait_read<1>();
+          named_bar_sync(1, 128);
+          if (leader) {
+            tma_reduce_add_3d(&tm_dqacc, buf, 32 * c4 + 16 * h, q0, bh);
+            bulk_commit();
+          }
         }
       }
     }
+    if (leader) bulk_wait_all();
   } else if (run && warp < 8) {
     // --------------------------------------------------------- P and dS
     const int wg = warp >> 2;
@@ -577,41 +613,49 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D, bool CAUSAL, bool DROPOUT>
 cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mdo, const BwdArgs& a, cudaStream_t st) {
+                            const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, cudaStream_t st) {
   using L = BwdLayout<D>;
+  static_assert(L::kSmem <= 232448, "shared memory budget");
   auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
-  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, a);
+  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, mdq, a);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_bwd_prepare(const BwdArgs& a, int d, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  const int npad = (a.N + 127) / 128 * 128;
+  if (d == 64)
+    bwd_pre_kernel<64><<<148 * 8, 256, 0, st>>>(a, BH, npad);
+  else
+    bwd_pre_kernel<128><<<148 * 8, 256, 0, st>>>(a, BH, npad);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const CUtensorMap& mdo, const BwdArgs& a, bool causal, bool dropout, cudaStream_t st) {
-  const int BH = a.B * a.H;
-  const int npad = (a.N + 127) / 128 * 128;
-  bwd_pre_kernel<D><<<148 * 8, 256, 0, st>>>(a, BH, npad);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+cudaError_t launch_bwd_recompute_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                   const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, bool causal,
+                                   bool dropout, cudaStream_t st) {
   if (causal)
-    e = dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, a, st)
-                : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, a, st);
-  else
-    e = dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, a, st)
-                : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, a, st);
-  if (e != cudaSuccess) return e;
-  const long long n8 = (long long)BH * a.N * D / 8;
-  bwd_post_kernel<<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, n8, a.scale);
-  return cudaGetLastError();
+    return dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, mdq, a, st)
+                   : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, mdq, a, st);
+  return dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, mdq, a, st)
+                 : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, mdq, a, st);
 }
 
-inline cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                              const CUtensorMap& mdo, const BwdArgs& a, int d, bool causal, bool dropout,
-                              cudaStream_t st) {
-  return d == 64 ? launch_bwd_d<64>(mq, mk, mv, mdo, a, causal, dropout, st)
-                 : launch_bwd_d<128>(mq, mk, mv, mdo, a, causal, dropout, st);
+inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                        const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, int d,
+                                        bool causal, bool dropout, cudaStream_t st) {
+  return d == 64 ? launch_bwd_recompute_d<64>(mq, mk, mv, mdo, mdq, a, causal, dropout, st)
+                 : launch_bwd_recompute_d<128>(mq, mk, mv, mdo, mdq, a, causal, dropout, st);
+}
+
+inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
+  const long long n8 = (long long)a.B * a.H * a.N * d / 8;
+  bwd_post_kernel<<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, n8, a.scale);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -45,6 +45,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Tensor map of the fp32 dQ accumulator [BH, N, d] written by 128-row x
+// 16-column reductions from 64-byte-swizzled staging tiles.
+int make_acc_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4u, (cuuint64_t)N * (cuuint64_t)d * 4u};
+  cuuint32_t box[3] = {16u, 128u, 1u};
+  cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
 // Tensor map of a [BH, N, d] bf16 tensor read in 128-row x 64-column boxes
 // with the 128-byte swizzle; rows past N read as zero.
 int make_tile_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
@@ -212,9 +228,92 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return fa::bwd_workspace_bytes(B * H, N, d);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-           void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p,
-           uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Checks shared by the backward entry points; fills the workspace pointers.
+int bwd_setup(int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, void* workspace,
+              size_t workspace_bytes, fa::BwdArgs* a) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc != FA_OK) return rc;
+  const size_t need = fa::bwd_workspace_bytes(B * H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
+  std::memset(a, 0, sizeof(*a));
+  a->B = B;
+  a->H = H;
+  a->N = N;
+  a->scale = scale;
+  a->scale_log2 = scale * 1.4426950408889634f;
+  a->drop_threshold = keep_threshold(dropout_p);
+  a->drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
+  a->seed = seed;
+  fa::bwd_workspace_split(workspace, B * H, N, d, &a->dq_acc, &a->lse2, &a->drow);
+  a->err = device_error_ptr();
+  if (!a->err) return cuda_fail(cudaErrorInvalidSymbol);
+  return FA_OK;
+}
+
+}  // namespace
+
+int fa_bwd_prepare(const void* o, const void* dout, const float* lse, int B, int H, int N, int d, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_common(B, H, N, d, 1.f, 0, 0.f);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!o || !dout || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  fa::BwdArgs a;
+  if ((rc = bwd_setup(B, H, N, d, 1.f, 0, 0.f, 0, workspace, workspace_bytes, &a)) != FA_OK) return rc;
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.lse = lse;
+  cudaError_t e = fa::launch_bwd_prepare(a, d, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
+                     int N, int d, float scale, int causal, float dropout_p, uint64_t seed, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !dout || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16))
+    return FA_ERR_ALIGNMENT;
+  fa::BwdArgs a;
+  if ((rc = bwd_setup(B, H, N, d, scale, causal, dropout_p, seed, workspace, workspace_bytes, &a)) != FA_OK)
+    return rc;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mdo, dout, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_acc_map(&mdq, a.dq_acc, B * H, N, d)) != FA_OK) return rc;
+  cudaError_t e = fa::launch_bwd_recompute(mq, mk, mv, mdo, mdq, a, d, causal != 0, dropout_p > 0.f,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  int rc = check_common(B, H, N, d, scale, 0, 0.f);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!dq) return FA_ERR_INVALID_ARG;
+  if (!aligned(dq, 16)) return FA_ERR_ALIGNMENT;
+  fa::BwdArgs a;
+  if ((rc = bwd_setup(B, H, N, d, scale, 0, 0.f, 0, workspace, workspace_bytes, &a)) != FA_OK) return rc;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  cudaError_t e = fa::launch_bwd_finalize(a, d, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+           void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -222,35 +321,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
-  const size_t need = fa::bwd_workspace_bytes(B * H, N, d);
-  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
-  CUtensorMap mq, mk, mv, mdo;
-  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mdo, dout, B * H, N, d)) != FA_OK) return rc;
-  fa::BwdArgs a;
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.scale = scale;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.drop_threshold = keep_threshold(dropout_p);
-  a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
-  a.seed = seed;
-  a.o = static_cast<const __nv_bfloat16*>(o);
-  a.dout = static_cast<const __nv_bfloat16*>(dout);
-  a.lse = lse;
-  a.dq = static_cast<__nv_bfloat16*>(dq);
-  a.dk = static_cast<__nv_bfloat16*>(dk);
-  a.dv = static_cast<__nv_bfloat16*>(dv);
-  fa::bwd_workspace_split(workspace, B * H, N, d, &a.dq_acc, &a.lse2, &a.drow);
-  a.err = device_error_ptr();
-  if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = fa::launch_bwd(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f, st);
-  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+  if ((rc = fa_bwd_prepare(o, dout, lse, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK) return rc;
+  if ((rc = fa_bwd_recompute(q, k, v, dout, dk, dv, B, H, N, d, scale, causal, dropout_p, seed, workspace,
+                             workspace_bytes, stream)) != FA_OK)
+    return rc;
+  return fa_bwd_finalize(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -81,6 +81,10 @@ __global__ void __launch_bounds__(320, 1)
 
   // Work tile.  For the causal mask the CTA with the most key tiles goes
   // first (longest-processing-time order across the grid).
+  // Work tile.  For the causal mask the CTA with the most key tiles goes
+  // first (longest-processing-time order across the grid); heads are
+  // interleaved, and the CTAs of a wave sweep the key tiles of their heads in
+  // near lockstep, so the K/V tiles they read stay in L2.
   const int BH = a.B * a.H;
   const int n_cta_tiles = (a.N + 255) >> 8;
   const int tile_rev = blockIdx.x / BH;
@@ -265,14 +269,28 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
         const bool last = j == nkv - 1;
-        // key 128 j + c is visible to query 128 (qt0 + t) + r iff c < lim
+        // key 128 j + c is visible to query 128 (qt0 + t) + r iff c < lim;
+        // only the diagonal tile (causal) or the ragged last tile masks
         int lim = 128;
-        if (CAUSAL && last) lim = r + 1;                          // diagonal tile
-        if (!CAUSAL && last && (a.N & 127)) lim = a.N - j * 128;  // padded keys past N
-        float mx = -INFINITY;
+        if (CAUSAL && last) lim = r + 1;
+        if (!CAUSAL && last && (a.N & 127)) lim = a.N - j * 128;
+        if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < lim) mx = fmaxf(mx, __uint_as_float(u[c >> 5][c & 31]));
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) u[c >> 5][c & 31] = 0xff800000u;  // -inf
+        }
+        // row maximum: four independent 3-input max chains
+        float mx4[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) mx4[g] = __uint_as_float(u[g][0]);
+#pragma unroll
+        for (int c = 1; c < 31; c += 2)
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            mx4[g] = max3(mx4[g], __uint_as_float(u[g][c]), __uint_as_float(u[g][c + 1]));
+#pragma unroll
+        for (int g = 0; g < 4; ++g) mx4[g] = fmaxf(mx4[g], __uint_as_float(u[g][31]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m_used, mx * sl2);
         if (__any_sync(0xffffffffu, m_new > m_used + 8.0f)) {
           const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
@@ -296,18 +314,30 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
+            if (__any_sync(0xffffffffu, lim < 128)) {
+#pragma unroll
+              for (int c = 0; c < 128; ++c)
+                if (c >= lim) u[c >> 5][c & 31] = 0xff800000u;
+            }
           }
         }
         const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-        float psum = 0.f;
+        // p = 2^(s * scale * log2 e - m): scale/subtract on the packed f32x2
+        // pipe, exponentials on MUFU, row sum in four packed accumulators
+        const uint64_t mul2 = f2_pack(sl2, sl2);
+        const uint64_t sub2 = f2_pack(-msub, -msub);
+        uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[4][16];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float x0 = 2 * c < lim ? __uint_as_float(u[(2 * c) >> 5][(2 * c) & 31]) : -INFINITY;
-          const float x1 = 2 * c + 1 < lim ? __uint_as_float(u[(2 * c + 1) >> 5][(2 * c + 1) & 31]) : -INFINITY;
-          float p0 = ex2(fmaf(x0, sl2, -msub));
-          float p1 = ex2(fmaf(x1, sl2, -msub));
-          psum += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[(2 * c) >> 5][(2 * c) & 31]),
+                                             __uint_as_float(u[(2 * c + 1) >> 5][(2 * c + 1) & 31])),
+                                     mul2, sub2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = ex2(x0);
+          float p1 = ex2(x1);
+          sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
           if (DROPOUT) {
             const uint32_t col = (uint32_t)(j * 128 + 2 * c);
             p0 = dropout_hash(rkey, col) >= a.drop_threshold ? p0 * a.drop_scale : 0.f;
@@ -315,7 +345,14 @@ __global__ void __launch_bounds__(320, 1)
           }
           pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
         }
-        l += psum;
+        {
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(sum2[0], s0, s1);
+          f2_unpack(sum2[1], s2, s3);
+          f2_unpack(sum2[2], s4, s5);
+          f2_unpack(sum2[3], s6, s7);
+          l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        }
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) tmem_st16(tS + 16u * c16, pk[c16]);
         tmem_st_wait();
