@@ -116,6 +116,30 @@ int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* wor
                     void* stream);
 
 /*
+ * fa_bwd without a caller-provided workspace.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory,
+ * such as plugin or custom-op interfaces that pass a kernel only its input
+ * and output tensors, or code that must not allocate at that point.
+ * Arguments, outputs and errors are those of fa_bwd; the scratch fa_bwd
+ * would take from `workspace` comes instead from a static device array of
+ * FA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  Nothing is allocated.
+ *  - Shapes whose fa_bwd_workspace_size exceeds FA_NOALLOC_SCRATCH_BYTES are
+ *    rejected with FA_ERR_TOO_LARGE before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array, which keeps whatever the
+ *    last call left in it (the backward clears what must start at zero).
+ *    Calls that overlap on the GPU, e.g. on two streams, race on it and
+ *    produce wrong results; serialise them.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                   float dropout_p, uint64_t seed, void* stream);
+
+/*
  * Debug export of the dropout mask: for each listed head bh = b*H + h
  * (heads[nheads]) and query row (rows[nrows]), writes the keep bit of every
  * key j < N to out[(hi * nrows + ri) * N + j] (1 = kept).  heads, rows and

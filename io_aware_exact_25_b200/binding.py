@@ -28,8 +28,10 @@ FA_ERR_DEVICE = -6
 FA_ERR_TOO_LARGE = -7
 
 EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
-           "fa_bwd_finalize", "fa_dropout_mask", "fa_strerror", "fa_last_cuda_error",
-           "fa_get_device_error", "fa_version")
+           "fa_bwd_finalize", "fa_bwd_noalloc", "fa_dropout_mask", "fa_strerror",
+           "fa_last_cuda_error", "fa_get_device_error", "fa_version")
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _lock = threading.Lock()
 _lib = None
@@ -59,12 +61,13 @@ def load() -> ctypes.CDLL:
         lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
         lib.fa_bwd_recompute.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
         lib.fa_bwd_finalize.argtypes = [vp, I, I, I, I, F, vp, SZ, vp]
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
         lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
-                   lib.fa_bwd_finalize, lib.fa_dropout_mask, lib.fa_get_device_error,
+                   lib.fa_bwd_finalize, lib.fa_bwd_noalloc, lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
         _lib = lib
@@ -166,6 +169,24 @@ def bwd_stages(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, s
                                _ptr(workspace), wsb, s), "fa_bwd_recompute")
     _call(lib.fa_bwd_finalize(_ptr(dq), B, H, N, d, float(scale), _ptr(workspace), wsb, s),
           "fa_bwd_finalize")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, causal=False, scale=None, dropout_p=0.0, seed=0,
+                stream=None):
+    """dQ, dK, dV via ``fa_bwd_noalloc`` into caller-provided outputs.
+
+    Uses the library's static scratch instead of a workspace, so nothing is
+    allocated here either (the outputs must be passed in).
+    """
+    _check_inputs(q, k, v, o, dout, dq, dk, dv)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, H, N, d, float(scale), int(bool(causal)), float(dropout_p),
+                               int(seed), _stream(stream))
+    _call(rc, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

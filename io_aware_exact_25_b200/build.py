@@ -8,7 +8,7 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfa_sm100.so")
-SOURCES = [os.path.join(PKG, "csrc", "fa_api.cu")]
+SOURCES = [os.path.join(PKG, "csrc", "fa_api.cu"), os.path.join(PKG, "csrc", "fa_noalloc.cu")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-shared"]
 
