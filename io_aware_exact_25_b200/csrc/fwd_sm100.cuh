@@ -19,7 +19,9 @@
 // column 128 t; P_t (bf16, 64 columns) overwrites the first half of S_t and is
 // the A operand of O_t += P_t V_j; O_t (fp32, D columns) at 256 + D t.
 // The two Q tiles ping-pong: while one tile's softmax runs, the tensor core
-// works on the other tile's MMAs.
+// works on the other tile's MMAs.  O_t is only rescaled by its own softmax
+// warps, after S_t(j) has completed, which implies that every earlier MMA of
+// the issuing thread -- O_t += P_t V(j-1) included -- has completed too.
 //
 // Online softmax in base 2: x = s * scale * log2(e); m is a running row
 // maximum that is only raised (and O, l rescaled) when the tile maximum
@@ -43,6 +45,10 @@ struct FwdArgs {
   int* err;          // device error word (may be null)
 };
 
+// Of every 8 pairs of probabilities, this many take the exponential on the
+// FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
+constexpr int kPolyPairsOf8 = 0;
+
 template <int D>
 struct FwdLayout {
   static constexpr int kThreads = 320;
@@ -52,7 +58,7 @@ struct FwdLayout {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + 2 * kTile;
   static constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
   static constexpr uint32_t kColO = 256;  // O_t at kColO + D * t
 };
@@ -74,7 +80,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bar_s = bar_kv_empty + L::kStages;          // [2]   S_t ready in TMEM
   uint64_t* bar_p = bar_s + 2;                          // [2]   P_t written (128 arrivals)
   uint64_t* bar_pv = bar_p + 2;                         // [2]   O_t += P_t V_j done
-  uint64_t* bar_drain = bar_pv + 2;                     //       all MMAs retired
+  uint64_t* bar_p_half = bar_pv + 2;                    // [2]   first half of P_t written
+  uint64_t* bar_drain = bar_p_half + 2;                 //       all MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   const uint32_t sbase = smem_u32(smem);
@@ -108,6 +115,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], 128);
       mbar_init(&bar_pv[t], 1);
+      mbar_init(&bar_p_half[t], 128);
     }
     mbar_init(bar_drain, 1);
     const bool misaligned = (sbase & 1023u) != 0u;
@@ -171,67 +179,86 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (run && warp == 8) {
     // ------------------------------------------------------- MMA issuer
+    // Issue order for key tile j: O0 += P0 V(j-1), S0(j), O1 += P1 V(j-1),
+    // S1(j).  S_t(j) overwrites the TMEM columns that hold P_t(j-1); it is
+    // queued directly behind the product that reads P_t(j-1) and the tensor
+    // core executes the MMAs of one issuing thread in order, so no wait is
+    // needed between them.  The softmax publishes P_t in two halves (keys
+    // 0-63, 64-127) so the product starts on the first half early.  K(j)
+    // sits at ring position 2j, V(j) at 2j+1; stages are released in ring
+    // order.
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // S = Q K^T, both K-major
       constexpr uint32_t kIdO = idesc_bf16(128, D, false, true);     // O += P V, V is MN-major
       bool ok = mbar_wait(&bar_q[0], 0, ab) && (!act1 || mbar_wait(&bar_q[1], 0, ab));
-      tc_fence_after();
-      int stage = 0;
-      uint32_t phase = 0;
       bool issued_any = false;
-      for (int j = 0; j < nkv_max && ok; ++j) {
-        // S_t = Q_t K_j^T
-        if (!mbar_wait(&bar_kv_full[stage], phase, ab)) break;
+      auto stage_of = [](int pos) { return pos % L::kStages; };
+      auto phase_of = [](int pos) { return (uint32_t)((pos / L::kStages) & 1); };
+      auto issue_s = [&](int t, uint32_t sK) {
+        const uint32_t sQ = sbase + L::kOffQ + t * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + 128u * t, desc_kmajor(sQ, kk, L::kHalf), desc_kmajor(sK, kk, L::kHalf), kIdS,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&bar_s[t]);
+        issued_any = true;
+      };
+      auto issue_pv = [&](int t, int j, uint32_t sV) -> bool {
+        if (!mbar_wait(&bar_p_half[t], j & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sK = sbase + L::kOffKV + stage * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        if (!mbar_wait(&bar_p[t], j & 1, ab)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk)
+          mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO, 1u);
+        mma_commit(&bar_pv[t]);
+        return true;
+      };
+      if (ok && mbar_wait(&bar_kv_full[0], 0, ab)) {
+        tc_fence_after();
+        const uint32_t sK0 = sbase + L::kOffKV;
+        issue_s(0, sK0);
+        if (nkv1 > 0) issue_s(1, sK0);
+        mma_commit(&bar_kv_empty[0]);
+      } else {
+        ok = false;
+      }
+      for (int j = 1; j < nkv_max && ok; ++j) {
+        const int posV = 2 * j - 1, posK = 2 * j;
+        if (!mbar_wait(&bar_kv_full[stage_of(posV)], phase_of(posV), ab) ||
+            !mbar_wait(&bar_kv_full[stage_of(posK)], phase_of(posK), ab))
+          break;
+        tc_fence_after();
+        const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTile;
+        const uint32_t sK = sbase + L::kOffKV + stage_of(posK) * L::kTile;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= (t ? nkv1 : nkv0)) continue;
-          // S_t shares its columns with P_t, which O_t += P_t V_{j-1} reads.
-          if (j > 0) {
-            if (!mbar_wait(&bar_pv[t], (j - 1) & 1, ab)) {
-              ok = false;
-              continue;
-            }
-            tc_fence_after();
-          }
-          const uint32_t sQ = sbase + L::kOffQ + t * L::kTile;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 128u * t, desc_kmajor(sQ, kk, L::kHalf), desc_kmajor(sK, kk, L::kHalf), kIdS,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(&bar_s[t]);
-          issued_any = true;
-        }
-        if (!ok) break;
-        mma_commit(&bar_kv_empty[stage]);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-        // O_t += P_t V_j
-        if (!mbar_wait(&bar_kv_full[stage], phase, ab)) break;
-        tc_fence_after();
-        const uint32_t sV = sbase + L::kOffKV + stage * L::kTile;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= (t ? nkv1 : nkv0)) continue;
-          if (!mbar_wait(&bar_p[t], j & 1, ab)) {
+          const int nkv_t = t ? nkv1 : nkv0;
+          if (!ok || j - 1 >= nkv_t) continue;
+          if (!issue_pv(t, j - 1, sV)) {
             ok = false;
             continue;
           }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bar_pv[t]);
+          if (j < nkv_t) issue_s(t, sK);
         }
         if (!ok) break;
-        mma_commit(&bar_kv_empty[stage]);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1u;
+        mma_commit(&bar_kv_empty[stage_of(posV)]);  // V(j-1) consumed
+        mma_commit(&bar_kv_empty[stage_of(posK)]);  // K(j) consumed
+      }
+      if (ok && nkv_max > 0) {
+        const int j = nkv_max - 1, posV = 2 * j + 1;
+        if (mbar_wait(&bar_kv_full[stage_of(posV)], phase_of(posV), ab)) {
+          tc_fence_after();
+          const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTile;
+          bool last_ok = true;
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (last_ok && j < (t ? nkv1 : nkv0)) last_ok = issue_pv(t, j, sV);
+          mma_commit(&bar_kv_empty[stage_of(posV)]);
         }
       }
       if (issued_any) {
@@ -333,10 +360,15 @@ __global__ void __launch_bounds__(320, 1)
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[(2 * c) >> 5][(2 * c) & 31]),
                                              __uint_as_float(u[(2 * c + 1) >> 5][(2 * c + 1) & 31])),
                                      mul2, sub2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = ex2(x0);
-          float p1 = ex2(x1);
+          float p0, p1;
+          if ((c & 7) < kPolyPairsOf8) {
+            exp2_poly_x2(x2, p0, p1);  // FMA pipe
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2(x0);  // MUFU
+            p1 = ex2(x1);
+          }
           sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
           if (DROPOUT) {
             const uint32_t col = (uint32_t)(j * 128 + 2 * c);
@@ -344,6 +376,14 @@ __global__ void __launch_bounds__(320, 1)
             p1 = dropout_hash(rkey, col + 1) >= a.drop_threshold ? p1 * a.drop_scale : 0.f;
           }
           pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
+          if (c == 31) {
+            // keys 0-63 done: publish them so O += P V can start
+            tmem_st16(tS, pk[0]);
+            tmem_st16(tS + 16u, pk[1]);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bar_p_half[t]);
+          }
         }
         {
           float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -353,8 +393,8 @@ __global__ void __launch_bounds__(320, 1)
           f2_unpack(sum2[3], s6, s7);
           l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         }
-#pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) tmem_st16(tS + 16u * c16, pk[c16]);
+        tmem_st16(tS + 32u, pk[2]);
+        tmem_st16(tS + 48u, pk[3]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar_p[t]);

@@ -386,6 +386,37 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for two values at once on the FMA pipe, for x <= 126 (x = -inf or
+// below -126 gives a value below 2^-125 instead of 0).  Cody-Waite split
+// x = n + f with n = round(x) and f in [-1/2, 1/2]: n comes from adding
+// 1.5 * 2^23 (the rounded integer lands in the low mantissa bits), 2^f from a
+// cubic, and n is added to the exponent field with integer arithmetic.  The
+// cubic is a relative-error minimax fit of 2^f on [-1/2, 1/2] computed for
+// this library (fp64 Remez exchange, coefficients rounded to fp32): max
+// relative error 7.5e-5, far below the bf16 resolution of the
+// probabilities it produces.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& r0, float& r1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));    // 1.5 * 2^23 + round(x)
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));   // round(x), exact
+  const uint64_t fr = f2_fma(n, f2_pack(-1.f, -1.f), xc);            // x - round(x), exact
+  uint64_t p = f2_fma(fr, f2_pack(0.0551716685295105f, 0.0551716685295105f),
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // low mantissa bits of t hold round(x); the high bits of t shifted by 23
+  // vanish mod 2^32, so t << 23 == round(x) << 23
+  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
