@@ -35,8 +35,9 @@
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
 // [0,32) and [64,96); R_dP [128,256) dP^T fp32, then dS^T bf16 in [128,160)
 // and [192,224), then the dQ partial (fp32, D columns); dV at 256, dK at
-// 256 + D.  MMA order per step: dP(i), dV(i), dK(i), S(i+1), dQ(i), so the
-// next step's softmax overlaps this step's dQ read-out.
+// 256 + D.  MMA order per step: dP(i), dV(i), dK(i), dQ(i), S(i+1); dP(i)
+// runs while the softmax warps form P(i), and the dQ read-out of one step
+// overlaps the next step's S and P.
 #pragma once
 
 #include "dropout_hash.cuh"
@@ -65,16 +66,21 @@ struct BwdArgs {
 
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace: the fp32 dQ accumulator over N rounded up to 128 rows, stored
+// tile by tile -- for each head, 128-row query tile and 16-column piece, one
+// contiguous 8 KB block of 128 rows x 16 columns whose 16-byte chunks are
+// permuted by the 64-byte swizzle (chunk k of row r at k ^ ((r >> 1) & 3)) --
+// then the scaled lse and D row vectors.
 inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   const size_t npad = round_up((size_t)N, 128);
-  return round_up((size_t)BH * N * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256);
+  return round_up((size_t)BH * npad * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256);
 }
 
 inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, float** lse2, float** drow) {
   const size_t npad = round_up((size_t)N, 128);
   char* p = static_cast<char*>(ws);
   *dq_acc = reinterpret_cast<float*>(p);
-  p += round_up((size_t)BH * N * d * 4, 256);
+  p += round_up((size_t)BH * npad * d * 4, 256);
   *lse2 = reinterpret_cast<float*>(p);
   p += round_up((size_t)BH * npad * 4, 256);
   *drow = reinterpret_cast<float*>(p);
@@ -82,8 +88,8 @@ inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, 
 
 // ------------------------------------------------------------ row pass
 
-// One warp per (padded) row: D_i = sum_c dO_ic O_ic in fp32, lse2_i, and the
-// row of the dQ accumulator set to zero.
+// One warp per (padded) row: D_i = sum_c dO_ic O_ic in fp32 and lse2_i; then
+// the whole dQ accumulator is set to zero.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, int npad) {
   constexpr int kPer = D / 32;  // elements per lane
@@ -102,12 +108,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
         const uint2 dv = *reinterpret_cast<const uint2*>(a.dout + off);
         acc = bf16_lo(ov.x) * bf16_lo(dv.x) + bf16_hi(ov.x) * bf16_hi(dv.x) + bf16_lo(ov.y) * bf16_lo(dv.y) +
               bf16_hi(ov.y) * bf16_hi(dv.y);
-        *reinterpret_cast<float4*>(a.dq_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         const uint32_t ov = *reinterpret_cast<const uint32_t*>(a.o + off);
         const uint32_t dv = *reinterpret_cast<const uint32_t*>(a.dout + off);
         acc = bf16_lo(ov) * bf16_lo(dv) + bf16_hi(ov) * bf16_hi(dv);
-        *reinterpret_cast<float2*>(a.dq_acc + off) = make_float2(0.f, 0.f);
       }
 #pragma unroll
       for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
@@ -120,15 +124,32 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
       a.lse2[r] = INFINITY;
     }
   }
+  const long long n4 = (long long)BH * npad * D / 4;
+  float4* acc4 = reinterpret_cast<float4*>(a.dq_acc);
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n4; u += (long long)gridDim.x * blockDim.x)
+    acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ = scale * accumulator, 8 elements per thread per iteration.
+// dQ = scale * accumulator, read from the tiled accumulator layout; each
+// thread converts 8 consecutive columns (two swizzled 16-byte chunks) of a row.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
-                                                       long long n8, float scale) {
+                                                       int BH, int N, float scale) {
+  const int npad = (N + 127) & ~127;
+  const long long n8 = (long long)BH * N * (D / 8);
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n8;
        u += (long long)gridDim.x * blockDim.x) {
-    const float4 x = reinterpret_cast<const float4*>(acc)[2 * u];
-    const float4 y = reinterpret_cast<const float4*>(acc)[2 * u + 1];
+    const int c8 = (int)(u % (D / 8));
+    const long long rowg = u / (D / 8);
+    const int bh = (int)(rowg / N);
+    const int i = (int)(rowg - (long long)bh * N);
+    const int tile = i >> 7, r = i & 127;
+    const int piece = c8 >> 1;            // 16-column piece
+    const int k0 = (c8 & 1) * 2;          // first of the two 4-column chunks
+    const int sw = (r >> 1) & 3;
+    const float* blk = acc + (((size_t)bh * (npad >> 7) + tile) * (D / 16) + piece) * 2048 + r * 16;
+    const float4 x = *reinterpret_cast<const float4*>(blk + ((k0 ^ sw) << 2));
+    const float4 y = *reinterpret_cast<const float4*>(blk + (((k0 + 1) ^ sw) << 2));
     uint4 w;
     w.x = pack_bf16x2(x.x * scale, x.y * scale);
     w.y = pack_bf16x2(x.z * scale, x.w * scale);
@@ -140,7 +161,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
 
 // ------------------------------------------------------- fused kernel
 
-template <int D>
+template <int D, bool DROPOUT>
 struct BwdLayout {
   static constexpr int kThreads = 448;
   static constexpr uint32_t kHalf = 128u * 128u;
@@ -152,12 +173,12 @@ struct BwdLayout {
   static constexpr uint32_t kOffQ = kOffV + kTile;
   static constexpr uint32_t kOffDO = kOffQ + kQStages * kTile;
   static constexpr uint32_t kOffDS = kOffDO + kDoStages * kTile;  // dS, 128 x 128 bf16, MN-major halves
-  static constexpr uint32_t kRowStage = 3u * 128u * 4u;             // lse2, D, dropout row keys
+  static constexpr uint32_t kRowStage = (DROPOUT ? 3u : 2u) * 128u * 4u;  // lse2, D (, dropout row keys)
   static constexpr uint32_t kOffRow = kOffDS + 2u * kHalf;
-  // dQ staging: three 128-row x 16-column fp32 pieces (64-byte rows,
-  // 64-byte swizzle), the source tiles of the TMA reductions
+  // dQ staging: 128-row x 16-column fp32 pieces (64-byte rows, 64-byte
+  // swizzle), each the source of one 8 KB bulk reduction
   static constexpr uint32_t kDqPiece = 128u * 64u;
-  static constexpr int kDqBufs = 3;
+  static constexpr int kDqBufs = (D == 128 && DROPOUT) ? 3 : 4;
   static constexpr uint32_t kOffDQ = kOffRow + 2u * kRowStage;
   static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
@@ -165,6 +186,7 @@ struct BwdLayout {
   static constexpr int kNumBars = 1 + 12 + 9;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
   static_assert(kOffDQ % 1024 == 0, "staging tiles must be swizzle-aligned");
+  static_assert(kSmem <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
@@ -176,8 +198,8 @@ template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_dqacc, const BwdArgs a) {
-  using L = BwdLayout<D>;
+               const BwdArgs a) {
+  using L = BwdLayout<D, DROPOUT>;
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -259,7 +281,6 @@ __global__ void __launch_bounds__(448, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_dqacc);
       mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
       for (int h = 0; h < D / 64; ++h) {
         tma_load_3d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, bh, bar_kv, pol_keep);
@@ -337,13 +358,19 @@ __global__ void __launch_bounds__(448, 1)
         mma_commit(bar_s);
         issued_any = true;
       }
+      // Per step: dP(i), dV(i), dK(i), dQ(i), S(i+1).  dP(i) overwrites the
+      // dQ(i-1) partial and waits for the dQ warpgroup to have read it; it then
+      // runs while the softmax warps form P(i).  dQ(i) overwrites the columns
+      // holding dS^T(i), which dK(i) reads, and S(i+1) those holding P^T(i),
+      // which dV(i) reads; each is queued behind its reader and the tensor core
+      // executes one thread's MMAs in order, so neither needs a wait.
       for (int it = 0; it < n_steps && ok; ++it) {
         const uint32_t ph = it & 1;
         const int qs = it & 1;
         const int ds_ = it % L::kDoStages;
         const uint32_t sQ = sbase + L::kOffQ + qs * L::kTile;
         const uint32_t sDO = sbase + L::kOffDO + ds_ * L::kTile;
-        // dP^T = V dO_i^T into R_dP (holds the previous dQ partial until read out)
+        // dP^T = V dO_i^T into R_dP
         if (!mbar_wait(&bar_do_full[ds_], (it / L::kDoStages) & 1, ab)) break;
         if (it > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab)) break;
         tc_fence_after();
@@ -359,7 +386,6 @@ __global__ void __launch_bounds__(448, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + L::kColDV, tmem + L::kColS + packed_col(kk), desc_mnmajor(sDO, kk, L::kHalf), kIdTM,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_dv);
         mma_commit(&bar_do_empty[ds_]);
         // dK += dS^T Q_i
         if (!mbar_wait(bar_ds, ph, ab)) break;
@@ -369,12 +395,17 @@ __global__ void __launch_bounds__(448, 1)
           mma_ts(tmem + L::kColDK, tmem + L::kColDP + packed_col(kk), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_dk);
+        // dQ_i partial = dS K_j into R_dP (behind dK, which read dS^T there)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar_dq);
         mma_commit(&bar_q_empty[qs]);
-        // S^T for the next step, once dV has consumed P^T from R_S
+        // S^T for the next step (behind dV, which read P^T from R_S)
         if (it + 1 < n_steps) {
           const int qn = (it + 1) & 1;
           if (!mbar_wait(&bar_q_full[qn], ((it + 1) >> 1) & 1, ab)) break;
-          if (!mbar_wait(bar_dv, ph, ab)) break;
           tc_fence_after();
           const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
 #pragma unroll
@@ -383,14 +414,6 @@ __global__ void __launch_bounds__(448, 1)
                    kk > 0 ? 1u : 0u);
           mma_commit(bar_s);
         }
-        // dQ_i partial = dS K_j into R_dP, once dK has consumed dS^T
-        if (!mbar_wait(bar_dk, ph, ab)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);
       }
       if (issued_any) {
         mma_commit(bar_drain);
@@ -418,15 +441,18 @@ __global__ void __launch_bounds__(448, 1)
       named_bar_sync(1, 128);
       if (*dq_flag == 0) break;
       tc_fence_after();
-      const int q0 = (i_begin + it) * 128;
+      float* acc_tile = a.dq_acc + ((size_t)bh * nT + (i_begin + it)) * (size_t)(128 * D);
+      // the whole row first, so the TMEM columns are released at once
+      uint32_t v[D / 32][32];
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) tmem_ld32(tQ + 32u * c4, v[c4]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) reg_fence(v[c4]);
+      tc_fence_before();
+      mbar_arrive(bar_dq_free);
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t v[32];
-        tmem_ld32_sync(tQ + 32u * c4, v);
-        if (c4 == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(bar_dq_free);
-        }
 #pragma unroll
         for (int h = 0; h < 2; ++h, ++piece) {
           const uint32_t buf = sbase + L::kOffDQ + (piece % L::kDqBufs) * L::kDqPiece;
@@ -434,14 +460,15 @@ __global__ void __launch_bounds__(448, 1)
           const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
-            st_shared_v4(rbase + (((uint32_t)q4 ^ sw) << 4), v[16 * h + 4 * q4], v[16 * h + 4 * q4 + 1],
-                         v[16 * h + 4 * q4 + 2], v[16 * h + 4 * q4 + 3]);
+            st_shared_v4(rbase + (((uint32_t)q4 ^ sw) << 4), v[c4][16 * h + 4 * q4], v[c4][16 * h + 4 * q4 + 1],
+                         v[c4][16 * h + 4 * q4 + 2], v[c4][16 * h + 4 * q4 + 3]);
           fence_proxy_async_smem();
-          // the tile the next piece writes was last read by piece - 2
-          if (leader) bulk_wait_read<1>();
+          // the staging tile the next piece writes was last read
+          // kDqBufs - 1 pieces ago
+          if (leader) bulk_wait_read<L::kDqBufs - 2>();
           named_bar_sync(1, 128);
           if (leader) {
-            tma_reduce_add_3d(&tm_dqacc, buf, 32 * c4 + 16 * h, q0, bh);
+            bulk_reduce_add_f32(acc_tile + (2 * c4 + h) * 2048, buf, L::kDqPiece);
             bulk_commit();
           }
         }
@@ -613,14 +640,13 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D, bool CAUSAL, bool DROPOUT>
 cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, cudaStream_t st) {
-  using L = BwdLayout<D>;
-  static_assert(L::kSmem <= 232448, "shared memory budget");
+                            const CUtensorMap& mdo, const BwdArgs& a, cudaStream_t st) {
+  using L = BwdLayout<D, DROPOUT>;
   auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
-  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, mdq, a);
+  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, a);
   return cudaGetLastError();
 }
 
@@ -636,25 +662,27 @@ inline cudaError_t launch_bwd_prepare(const BwdArgs& a, int d, cudaStream_t st) 
 
 template <int D>
 cudaError_t launch_bwd_recompute_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                   const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, bool causal,
+                                   const CUtensorMap& mdo, const BwdArgs& a, bool causal,
                                    bool dropout, cudaStream_t st) {
   if (causal)
-    return dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, mdq, a, st)
-                   : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, mdq, a, st);
-  return dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, mdq, a, st)
-                 : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, mdq, a, st);
+    return dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, a, st)
+                   : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, a, st);
+  return dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, a, st)
+                 : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, a, st);
 }
 
 inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                        const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a, int d,
+                                        const CUtensorMap& mdo, const BwdArgs& a, int d,
                                         bool causal, bool dropout, cudaStream_t st) {
-  return d == 64 ? launch_bwd_recompute_d<64>(mq, mk, mv, mdo, mdq, a, causal, dropout, st)
-                 : launch_bwd_recompute_d<128>(mq, mk, mv, mdo, mdq, a, causal, dropout, st);
+  return d == 64 ? launch_bwd_recompute_d<64>(mq, mk, mv, mdo, a, causal, dropout, st)
+                 : launch_bwd_recompute_d<128>(mq, mk, mv, mdo, a, causal, dropout, st);
 }
 
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
-  const long long n8 = (long long)a.B * a.H * a.N * d / 8;
-  bwd_post_kernel<<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, n8, a.scale);
+  if (d == 64)
+    bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.N, a.scale);
+  else
+    bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.N, a.scale);
   return cudaGetLastError();
 }
 

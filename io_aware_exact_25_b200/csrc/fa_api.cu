@@ -45,22 +45,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map of the fp32 dQ accumulator [BH, N, d] written by 128-row x
-// 16-column reductions from 64-byte-swizzled staging tiles.
-int make_acc_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return cuda_fail(cudaErrorNotSupported);
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 4u, (cuuint64_t)N * (cuuint64_t)d * 4u};
-  cuuint32_t box[3] = {16u, 128u, 1u};
-  cuuint32_t estride[3] = {1u, 1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-  return FA_OK;
-}
-
 // Tensor map of a [BH, N, d] bf16 tensor read in 128-row x 64-column boxes
 // with the 128-byte swizzle; rows past N read as zero.
 int make_tile_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
@@ -286,13 +270,12 @@ int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* do
     return rc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo;
   if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
   if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
   if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
   if ((rc = make_tile_map(&mdo, dout, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_acc_map(&mdq, a.dq_acc, B * H, N, d)) != FA_OK) return rc;
-  cudaError_t e = fa::launch_bwd_recompute(mq, mk, mv, mdo, mdq, a, d, causal != 0, dropout_p > 0.f,
+  cudaError_t e = fa::launch_bwd_recompute(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }

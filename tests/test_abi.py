@@ -94,7 +94,7 @@ def test_workspace_size_formula(lib, B, H, N, d):
 
     def up(x):
         return (x + 255) // 256 * 256
-    expect = up(B * H * N * d * 4) + 2 * up(B * H * npad * 4)
+    expect = up(B * H * npad * d * 4) + 2 * up(B * H * npad * 4)
     assert lib.fa_bwd_workspace_size(B, H, N, d) == expect
     assert lib.fa_bwd_workspace_size(B, H, N, 96) == 0
     assert lib.fa_bwd_workspace_size(0, H, N, d) == 0
