@@ -194,6 +194,10 @@ struct BwdLayout {
 // two P/dS warpgroups: queries 0-63 at [0,32), 64-127 at [64,96).
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
 
+// Of every 8 pairs of recomputed probabilities, this many take the
+// exponential on the FMA pipe (polynomial), the rest on MUFU.
+constexpr int kBwdPolyPairsOf8 = 0;
+
 template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -507,16 +511,28 @@ __global__ void __launch_bounds__(448, 1)
       tmem_ld_wait();
       reg_fence(u[0]);
       reg_fence(u[1]);
-      // P^T_jq = 2^(s * scale * log2 e - lse2_q); padded queries have lse2 = +inf
+      // P^T_jq = 2^(s * scale * log2 e - lse2_q); padded queries have lse2 = +inf.
+      // Scale/subtract on the packed f32x2 pipe; of every 8 pairs,
+      // kBwdPolyPairsOf8 take the exponential on the FMA pipe (polynomial),
+      // the rest on MUFU.
       float p[64];
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l4 = ld_shared_f4(rowbuf + 4u * (col0 + 4 * c4));
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;
-          p[c] = ex2(fmaf(__uint_as_float(u[c >> 5][c & 31]), sl2, -lv[e]));
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int c = 4 * c4 + 2 * e2;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[c >> 5][c & 31]), __uint_as_float(u[c >> 5][(c + 1) & 31])),
+                                     sl2x2, f2_pack(e2 ? -l4.z : -l4.x, e2 ? -l4.w : -l4.y));
+          if (((c >> 1) & 7) < kBwdPolyPairsOf8) {
+            exp2_poly_x2(x2, p[c], p[c + 1]);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p[c] = ex2(x0);
+            p[c + 1] = ex2(x1);
+          }
         }
       }
       if (!key_ok) {
@@ -579,17 +595,21 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int c2 = 0; c2 < 8; ++c2) {
           const float4 d4 = ld_shared_f4(rowbuf + 512u + 4u * (col0 + 32 * hf + 4 * c2));
-          const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-          float ds[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 32 * hf + 4 * c2 + e;
-            float dp = __uint_as_float(g[4 * c2 + e]);
-            if (DROPOUT) dp = ((keep_bits[c >> 5] >> (c & 31)) & 1u) ? dp * a.drop_scale : 0.f;
-            ds[e] = p[c] * (dp - dv[e]);
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = 32 * hf + 4 * c2 + 2 * e2;
+            float dp0 = __uint_as_float(g[4 * c2 + 2 * e2]), dp1 = __uint_as_float(g[4 * c2 + 2 * e2 + 1]);
+            if (DROPOUT) {
+              dp0 = ((keep_bits[c >> 5] >> (c & 31)) & 1u) ? dp0 * a.drop_scale : 0.f;
+              dp1 = ((keep_bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? dp1 * a.drop_scale : 0.f;
+            }
+            // dS = P * (dP - D) = P * dP - P * D on the packed pipe
+            const uint64_t p2 = f2_pack(p[c], p[c + 1]);
+            const uint64_t pd = f2_mul(p2, f2_pack(e2 ? -d4.z : -d4.x, e2 ? -d4.w : -d4.y));
+            float ds0, ds1;
+            f2_unpack(f2_fma(p2, f2_pack(dp0, dp1), pd), ds0, ds1);
+            pk[2 * c2 + e2] = pack_bf16x2(ds0, ds1);
           }
-          pk[2 * c2] = pack_bf16x2(ds[0], ds[1]);
-          pk[2 * c2 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
         tmem_st16(tDSst + 16u * hf, pk);
         // shared-memory copy (A operand of dQ = dS K): row jr of this half,

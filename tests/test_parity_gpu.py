@@ -31,7 +31,8 @@ def _check(name, got, ref, exclude_rows=None):
     absolute bound, so the bound there is one ulp (2^-8 |ref|).  Rows listed
     in ``exclude_rows`` (index into axis -2) are left out of the relative
     metric only: they are rows whose exact value is identically zero, where a
-    relative error is undefined; they still meet the absolute bound.
+    relative error is undefined; they still meet the absolute bound.  For the
+    same reason an all-zero reference is held to the absolute bound only.
     """
     g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
     assert np.all(np.isfinite(g)), f"{name}: non-finite output"
@@ -43,7 +44,9 @@ def _check(name, got, ref, exclude_rows=None):
         keep = np.ones(ref.shape[-2], bool)
         keep[list(exclude_rows)] = False
         g, ref = g[..., keep, :], ref[..., keep, :]
-    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
+    if np.linalg.norm(ref) == 0.0:
+        return  # exactly zero (e.g. every row sees a single key): relative error undefined
+    rel = np.linalg.norm(g - ref) / np.linalg.norm(ref)
     assert rel <= REL_L2, f"{name}: rel L2 err {rel:.3e}"
 
 
