@@ -333,11 +333,10 @@ def run_ours(args, w):
     e2e_ms = e0.elapsed_time(e1)
 
     # max over ranks
-    times = torch.tensor([elapsed_ms, e2e_ms] + per_stage_ms, dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(times[0]), float(times[1])
-    per_stage_ms = [float(t) for t in times[2:]]
+    from io_aware_exact_25_b200.replicas import max_over_ranks
+    times = max_over_ranks([elapsed_ms, e2e_ms] + per_stage_ms, device=dev)
+    elapsed_ms, e2e_ms = times[0], times[1]
+    per_stage_ms = times[2:]
 
     if rank == 0:
         ff, fb = w.fwd_flops(), w.bwd_flops()
