@@ -174,12 +174,14 @@ struct BwdLayout {
   static constexpr uint32_t kOffDO = kOffQ + kQStages * kTile;
   static constexpr uint32_t kOffDS = kOffDO + kDoStages * kTile;  // dS, 128 x 128 bf16, MN-major halves
   static constexpr uint32_t kRowStage = (DROPOUT ? 3u : 2u) * 128u * 4u;  // lse2, D (, dropout row keys)
+  // double-buffered row statistics, except where shared memory runs out
+  static constexpr int kRowStages = (D == 128 && DROPOUT) ? 1 : 2;
   static constexpr uint32_t kOffRow = kOffDS + 2u * kHalf;
   // dQ staging: 128-row x 16-column fp32 pieces (64-byte rows, 64-byte
   // swizzle), each the source of one 8 KB bulk reduction
   static constexpr uint32_t kDqPiece = 128u * 64u;
-  static constexpr int kDqBufs = (D == 128 && DROPOUT) ? 3 : 4;
-  static constexpr uint32_t kOffDQ = kOffRow + 2u * kRowStage;
+  static constexpr int kDqBufs = 4;
+  static constexpr uint32_t kOffDQ = (kOffRow + kRowStages * kRowStage + 1023u) & ~1023u;
   static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
   // row_empty[2], s, dp, p, ds, dv, dk, dq, dq_free, drain
@@ -317,8 +319,8 @@ __global__ void __launch_bounds__(448, 1)
       }
       ++do_issued;
       // row statistics of query tile i
-      const int rs = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_row_empty[rs], ((it >> 1) & 1) ^ 1u, ab))) {
+      const int rs = it % L::kRowStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_row_empty[rs], ((it / L::kRowStages) & 1) ^ 1u, ab))) {
         ok = false;
         break;
       }
@@ -428,54 +430,92 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------ dQ read-out + accumulate
     // The partial dQ_i (128 rows x D fp32, query rows on the TMEM lanes) is
     // added into the fp32 accumulator in 16-column pieces: every thread
-    // writes its row of the piece into a 64-byte-swizzled staging tile, and
-    // one thread issues a tiled TMA reduction of the whole 128 x 16 tile.
-    // Three staging tiles rotate; a tile is rewritten only after the
-    // reduction issued from it three pieces earlier has read it.  The loop is
-    // uniform over the warpgroup (one thread waits, a named barrier shares
-    // the outcome), so every thread reaches every named barrier.
+    // writes its row of a piece into a 64-byte-swizzled staging tile, and
+    // one thread adds each whole 8 KB tile with a bulk reduction.  With four
+    // staging tiles, the first 64 columns are staged while the rest is still
+    // being read from TMEM; the TMEM columns are released as soon as the whole
+    // row is in registers or shared memory, before any reduction waits.  The
+    // loop is uniform over the warpgroup (one thread waits, a named barrier
+    // shares the outcome), so every thread reaches every named barrier.
+    static_assert(D == 64 || L::kDqBufs >= 4, "staging tiles");
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query within the tile == TMEM lane
     const bool leader = warp == 8 && lane == 0;
     const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDP;
+    const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
     volatile int* dq_flag = abort_flag + 1;
-    uint32_t piece = 0;
+    // stage 32 columns (two 16-column pieces) of this row into tiles t, t+1
+    auto stage = [&](const uint32_t (&v)[32], int t) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t rbase = sbase + L::kOffDQ + (uint32_t)(t + h) * L::kDqPiece + (uint32_t)row * 64u;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_shared_v4(rbase + (((uint32_t)q4 ^ sw) << 4), v[16 * h + 4 * q4], v[16 * h + 4 * q4 + 1],
+                       v[16 * h + 4 * q4 + 2], v[16 * h + 4 * q4 + 3]);
+      }
+    };
+    // after a named barrier: add staging tiles 0..n-1 into pieces p0..p0+n-1
+    auto reduce = [&](float* acc_tile, int p0, int n) {
+      if (leader) {
+        for (int t = 0; t < n; ++t)
+          bulk_reduce_add_f32(acc_tile + (p0 + t) * 2048, sbase + L::kOffDQ + (uint32_t)t * L::kDqPiece, L::kDqPiece);
+        bulk_commit();
+      }
+    };
     for (int it = 0; it < n_steps; ++it) {
-      if (leader) *dq_flag = mbar_wait(bar_dq, it & 1, ab) ? 1 : 0;
+      // the staging tiles are free once the previous step's reductions read them
+      if (leader) {
+        bulk_wait_read<0>();
+        *dq_flag = mbar_wait(bar_dq, it & 1, ab) ? 1 : 0;
+      }
       named_bar_sync(1, 128);
       if (*dq_flag == 0) break;
       tc_fence_after();
       float* acc_tile = a.dq_acc + ((size_t)bh * nT + (i_begin + it)) * (size_t)(128 * D);
-      // the whole row first, so the TMEM columns are released at once
-      uint32_t v[D / 32][32];
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) tmem_ld32(tQ + 32u * c4, v[c4]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) reg_fence(v[c4]);
-      tc_fence_before();
-      mbar_arrive(bar_dq_free);
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h, ++piece) {
-          const uint32_t buf = sbase + L::kOffDQ + (piece % L::kDqBufs) * L::kDqPiece;
-          const uint32_t rbase = buf + (uint32_t)row * 64u;
-          const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            st_shared_v4(rbase + (((uint32_t)q4 ^ sw) << 4), v[c4][16 * h + 4 * q4], v[c4][16 * h + 4 * q4 + 1],
-                         v[c4][16 * h + 4 * q4 + 2], v[c4][16 * h + 4 * q4 + 3]);
-          fence_proxy_async_smem();
-          // the staging tile the next piece writes was last read
-          // kDqBufs - 1 pieces ago
-          if (leader) bulk_wait_read<L::kDqBufs - 2>();
-          named_bar_sync(1, 128);
-          if (leader) {
-            bulk_reduce_add_f32(acc_tile + (2 * c4 + h) * 2048, buf, L::kDqPiece);
-            bulk_commit();
-          }
+      if (D == 64) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tQ, v0);
+        tmem_ld32(tQ + 32u, v1);
+        tmem_ld_wait();
+        reg_fence(v0);
+        reg_fence(v1);
+        tc_fence_before();
+        mbar_arrive(bar_dq_free);
+        stage(v0, 0);
+        stage(v1, 2);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        reduce(acc_tile, 0, 4);
+      } else {
+        {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tQ, v0);
+          tmem_ld32(tQ + 32u, v1);
+          tmem_ld_wait();
+          reg_fence(v0);
+          reg_fence(v1);
+          stage(v0, 0);
+          stage(v1, 2);
         }
+        uint32_t v2[32], v3[32];
+        tmem_ld32(tQ + 64u, v2);
+        tmem_ld32(tQ + 96u, v3);
+        tmem_ld_wait();
+        reg_fence(v2);
+        reg_fence(v3);
+        tc_fence_before();
+        mbar_arrive(bar_dq_free);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        reduce(acc_tile, 0, 4);
+        if (leader) bulk_wait_read<0>();
+        named_bar_sync(1, 128);
+        stage(v2, 0);
+        stage(v3, 2);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        reduce(acc_tile, 4, 4);
       }
     }
     if (leader) bulk_wait_all();
@@ -498,9 +538,9 @@ __global__ void __launch_bounds__(448, 1)
     for (int it = 0; it < n_steps; ++it) {
       const int i = i_begin + it;
       const uint32_t ph = it & 1;
-      const int rs = it & 1;
+      const int rs = it % L::kRowStages;
       const uint32_t rowbuf = sbase + L::kOffRow + rs * L::kRowStage;
-      if (!mbar_wait(bar_s, ph, ab) || !mbar_wait(&bar_row_full[rs], (it >> 1) & 1, ab)) {
+      if (!mbar_wait(bar_s, ph, ab) || !mbar_wait(&bar_row_full[rs], (it / L::kRowStages) & 1, ab)) {
         ok = false;
         break;
       }
