@@ -616,7 +616,16 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_before();
         mbar_arrive(bar_p);
       }
-      // dS^T = P^T * (dP^T * Z / (1 - p) - D), two 32-column halves
+      // the undropped P^T for dS, as fp16 pairs (relative error 2^-11, below
+      // the bf16 rounding dS itself gets): frees registers so both dP halves
+      // load with one wait
+      uint32_t ph16[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        __half2 hv = __floats2half2_rn(p[2 * c], p[2 * c + 1]);
+        ph16[c] = *reinterpret_cast<uint32_t*>(&hv);
+      }
+      // dS^T = P^T * (dP^T * Z / (1 - p) - D)
       if (!mbar_wait(bar_dp, ph, ab)) {
         ok = false;
         break;
@@ -627,10 +636,14 @@ __global__ void __launch_bounds__(448, 1)
         break;
       }
       tc_fence_after();
+      uint32_t g[2][32];
+      tmem_ld32(tDP, g[0]);
+      tmem_ld32(tDP + 32u, g[1]);
+      tmem_ld_wait();
+      reg_fence(g[0]);
+      reg_fence(g[1]);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        uint32_t g[32];
-        tmem_ld32_sync(tDP + 32u * hf, g);
         uint32_t pk[16];
 #pragma unroll
         for (int c2 = 0; c2 < 8; ++c2) {
@@ -638,13 +651,14 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int c = 32 * hf + 4 * c2 + 2 * e2;
-            float dp0 = __uint_as_float(g[4 * c2 + 2 * e2]), dp1 = __uint_as_float(g[4 * c2 + 2 * e2 + 1]);
+            float dp0 = __uint_as_float(g[hf][4 * c2 + 2 * e2]), dp1 = __uint_as_float(g[hf][4 * c2 + 2 * e2 + 1]);
             if (DROPOUT) {
               dp0 = ((keep_bits[c >> 5] >> (c & 31)) & 1u) ? dp0 * a.drop_scale : 0.f;
               dp1 = ((keep_bits[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? dp1 * a.drop_scale : 0.f;
             }
             // dS = P * (dP - D) = P * dP - P * D on the packed pipe
-            const uint64_t p2 = f2_pack(p[c], p[c + 1]);
+            const float2 pf = __half22float2(*reinterpret_cast<const __half2*>(&ph16[c >> 1]));
+            const uint64_t p2 = f2_pack(pf.x, pf.y);
             const uint64_t pd = f2_mul(p2, f2_pack(e2 ? -d4.z : -d4.x, e2 ? -d4.w : -d4.y));
             float ds0, ds1;
             f2_unpack(f2_fma(p2, f2_pack(dp0, dp1), pd), ds0, ds1);
