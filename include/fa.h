@@ -70,6 +70,27 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            float scale, int causal, float dropout_p, uint64_t seed, void* stream);
 
 /*
+ * Element strides of one logical [B, H, N, d] bf16 tensor whose last (d)
+ * dimension is contiguous: element (b, h, n, c) is at base[b*b_ + h*h_ +
+ * n*n_ + c] with b_ = .b, h_ = .h, n_ = .n.  Every stride times 2 bytes must be
+ * a multiple of 16.  Dense [B,H,N,d] is {H*N*d, N*d, d}; the pages' API layout
+ * (batch, seq_len, num_heads, head_dim) ("FlashAttention for Efficient
+ * Training", Integration with Frameworks) is {N*H*d, d, H*d}.
+ */
+typedef struct fa_strides {
+  int64_t b, h, n;
+} fa_strides;
+
+/*
+ * fa_fwd on strided tensors: strides[4] for q, k, v, o in that order (lse
+ * stays a dense fp32 [B,H,N]).  Errors as fa_fwd; FA_ERR_ALIGNMENT for a
+ * stride that breaks 16-byte row alignment.
+ */
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                   int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                   void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this shape: an fp32 dQ
  * accumulator [B,H,N,d] plus two fp32 row vectors (scaled lse and
  * D_i = dO_i . O_i) padded to a multiple of 128 rows.  Returns 0 for an empty
@@ -94,6 +115,15 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p,
            uint64_t seed, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd on strided tensors: strides[8] for q, k, v, o, dout, dq, dk, dv in
+ * that order (lse dense).  Errors as fa_bwd.
+ */
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d, float scale,
+                   int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 /*
  * The three stages fa_bwd runs, callable one by one on the same stream (for

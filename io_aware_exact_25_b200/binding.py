@@ -27,7 +27,7 @@ FA_ERR_CUDA = -5
 FA_ERR_DEVICE = -6
 FA_ERR_TOO_LARGE = -7
 
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
+EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -35,6 +35,11 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _lock = threading.Lock()
 _lib = None
+
+
+class FaStrides(ctypes.Structure):
+    """Element strides (batch, head, row) of a [B,H,N,d] tensor, d contiguous."""
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("n", ctypes.c_int64)]
 
 
 class FaError(RuntimeError):
@@ -55,6 +60,10 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         vp, I, F, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
+        SP = ctypes.POINTER(FaStrides)
+        lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp]
+        lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, SZ,
+                                       vp]
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
@@ -66,7 +75,7 @@ def load() -> ctypes.CDLL:
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
-        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
+        for fn in (lib.fa_fwd, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
                    lib.fa_bwd_finalize, lib.fa_bwd_noalloc, lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
@@ -89,15 +98,30 @@ def _ptr(t) -> int | None:
 
 
 def _check_inputs(*ts):
+    """[B,H,N,d] bf16 CUDA tensors (any strides with a contiguous last dim)."""
+    shape = ts[0].shape
     for t in ts:
         if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors (there is no CPU path)")
         if t.dtype != torch.bfloat16:
             raise ValueError("q, k, v, o, dO must be bf16")
+        if t.dim() != 4 or t.shape != shape:
+            raise ValueError("tensors must be [B,H,N,d] of one shape")
+        if t.stride(-1) != 1:
+            raise ValueError("the head dimension must be contiguous")
+
+
+def _check_dense(*ts):
+    for t in ts:
         if not t.is_contiguous():
-            raise ValueError("tensors must be contiguous [B,H,N,d]")
-        if t.dim() != 4:
-            raise ValueError("tensors must be [B,H,N,d]")
+            raise ValueError("this entry point takes dense [B,H,N,d] tensors")
+
+
+def _strides(*ts):
+    arr = (FaStrides * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = FaStrides(t.stride(0), t.stride(1), t.stride(2))
+    return arr
 
 
 def _call(rc: int, what: str):
@@ -115,8 +139,9 @@ def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=No
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    rc = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
-                       int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
+    _check_inputs(q, o)
+    rc = load().fa_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _strides(q, k, v, o), B, H, N, d,
+                               float(scale), int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
     _call(rc, "fa_fwd")
     return o, lse
 
@@ -138,18 +163,21 @@ def bwd(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, 
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    rc = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
-                       _ptr(dv), B, H, N, d, float(scale), int(bool(causal)), float(dropout_p), int(seed),
-                       _ptr(workspace), int(workspace.numel() * workspace.element_size()),
-                       _stream(stream))
+    _check_inputs(q, dq, dk, dv)
+    rc = load().fa_bwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _strides(q, k, v, o, dout, dq, dk, dv), B, H, N, d, float(scale),
+                               int(bool(causal)), float(dropout_p), int(seed), _ptr(workspace),
+                               int(workspace.numel() * workspace.element_size()), _stream(stream))
     _call(rc, "fa_bwd")
     return dq, dk, dv
 
 
 def bwd_stages(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, dq=None,
                dk=None, dv=None, workspace=None, stream=None):
-    """The backward as its three C-ABI stages (prepare, recompute, finalize)."""
+    """The backward as its three C-ABI stages (prepare, recompute, finalize);
+    dense [B,H,N,d] tensors only."""
     _check_inputs(q, k, v, o, dout)
+    _check_dense(q, k, v, o, dout)
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -180,6 +208,7 @@ def bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, causal=False, scale=None, dro
     allocated here either (the outputs must be passed in).
     """
     _check_inputs(q, k, v, o, dout, dq, dk, dv)
+    _check_dense(q, k, v, o, dout, dq, dk, dv)
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)

@@ -52,12 +52,19 @@ struct BwdArgs {
   uint32_t drop_threshold;
   float drop_scale;
   uint64_t seed;
+  // bf16 [B,H,N,D] tensors with element strides (batch, head, row); D is
+  // contiguous
   const __nv_bfloat16* o;
+  long long o_sb, o_sh, o_sn;
   const __nv_bfloat16* dout;
-  const float* lse;  // [BH, N] natural log
+  long long do_sb, do_sh, do_sn;
+  const float* lse;  // [BH, N] contiguous, natural log
   __nv_bfloat16* dq;
+  long long dq_sb, dq_sh, dq_sn;
   __nv_bfloat16* dk;
+  long long dk_sb, dk_sh, dk_sn;
   __nv_bfloat16* dv;
+  long long dv_sb, dv_sh, dv_sn;
   float* dq_acc;  // [BH, N, D] fp32 scratch
   float* lse2;    // [BH, Npad] scratch: lse * log2(e), +inf on padded rows
   float* drow;    // [BH, Npad] scratch: D_i, 0 on padded rows
@@ -101,16 +108,18 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
     const int bh = (int)(r / npad);
     const int i = (int)(r - (long long)bh * npad);
     if (i < a.N) {
-      const size_t off = ((size_t)bh * a.N + i) * D + lane * kPer;
+      const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+      const __nv_bfloat16* orow = a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + lane * kPer;
+      const __nv_bfloat16* drow = a.dout + b_ * a.do_sb + h_ * a.do_sh + (long long)i * a.do_sn + lane * kPer;
       float acc = 0.f;
       if (kPer == 4) {
-        const uint2 ov = *reinterpret_cast<const uint2*>(a.o + off);
-        const uint2 dv = *reinterpret_cast<const uint2*>(a.dout + off);
+        const uint2 ov = *reinterpret_cast<const uint2*>(orow);
+        const uint2 dv = *reinterpret_cast<const uint2*>(drow);
         acc = bf16_lo(ov.x) * bf16_lo(dv.x) + bf16_hi(ov.x) * bf16_hi(dv.x) + bf16_lo(ov.y) * bf16_lo(dv.y) +
               bf16_hi(ov.y) * bf16_hi(dv.y);
       } else {
-        const uint32_t ov = *reinterpret_cast<const uint32_t*>(a.o + off);
-        const uint32_t dv = *reinterpret_cast<const uint32_t*>(a.dout + off);
+        const uint32_t ov = *reinterpret_cast<const uint32_t*>(orow);
+        const uint32_t dv = *reinterpret_cast<const uint32_t*>(drow);
         acc = bf16_lo(ov) * bf16_lo(dv) + bf16_hi(ov) * bf16_hi(dv);
       }
 #pragma unroll
@@ -134,7 +143,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
 // thread converts 8 consecutive columns (two swizzled 16-byte chunks) of a row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
-                                                       int BH, int N, float scale) {
+                                                       int BH, int H, int N, long long sb, long long sh, long long sn,
+                                                       float scale) {
   const int npad = (N + 127) & ~127;
   const long long n8 = (long long)BH * N * (D / 8);
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n8;
@@ -155,7 +165,8 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     w.y = pack_bf16x2(x.z * scale, x.w * scale);
     w.z = pack_bf16x2(y.x * scale, y.y * scale);
     w.w = pack_bf16x2(y.z * scale, y.w * scale);
-    reinterpret_cast<uint4*>(dq)[u] = w;
+    const int b_ = bh / H, h_ = bh - b_ * H;
+    *reinterpret_cast<uint4*>(dq + b_ * sb + h_ * sh + (long long)i * sn + 8 * c8) = w;
   }
 }
 
@@ -240,6 +251,7 @@ __global__ void __launch_bounds__(448, 1)
   // and accumulator rows they share stay in L2.
   const int jt = blockIdx.x / BH;  // key tile
   const int bh = blockIdx.x - jt * BH;
+  const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
   const int i_begin = CAUSAL ? jt : 0;
   const int n_steps = nT - i_begin;
   const int npad = nT * 128;
@@ -289,8 +301,8 @@ __global__ void __launch_bounds__(448, 1)
       prefetch_tmap(&tm_do);
       mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
       for (int h = 0; h < D / 64; ++h) {
-        tma_load_3d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, bh, bar_kv, pol_keep);
-        tma_load_3d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, jt * 128, bh, bar_kv, pol_keep);
+        tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, hh, bb, bar_kv, pol_keep);
+        tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, jt * 128, hh, bb, bar_kv, pol_keep);
       }
     }
     // All 32 lanes run this loop (they compute the dropout row keys); the
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(448, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, bh,
+          tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, hh, bb,
                       &bar_q_full[qs], pol_keep);
       }
       ++q_issued;
@@ -314,7 +326,7 @@ __global__ void __launch_bounds__(448, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar_do_full[ds_], L::kTile);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, bh,
+          tma_load_4d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, hh, bb,
                       &bar_do_full[ds_], pol_keep);
       }
       ++do_issued;
@@ -328,7 +340,7 @@ __global__ void __launch_bounds__(448, 1)
       if (DROPOUT) {
         uint32_t* keys = reinterpret_cast<uint32_t*>(rowbuf + 2 * 512);
         for (int c = lane; c < 128; c += 32)
-          keys[c] = dropout_row_key(a.seed, (uint32_t)(bh / a.H), (uint32_t)(bh % a.H), (uint32_t)(i * 128 + c));
+          keys[c] = dropout_row_key(a.seed, (uint32_t)bb, (uint32_t)hh, (uint32_t)(i * 128 + c));
         __syncwarp();
       }
       if (lane == 0) {
@@ -686,7 +698,8 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_after();
       const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
       const float mul = wg == 0 ? 1.f : a.scale;
-      __nv_bfloat16* dst = (wg == 0 ? a.dv : a.dk) + ((size_t)bh * a.N + (size_t)(key_ok ? key : 0)) * D;
+      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + (long long)(key_ok ? key : 0) * a.dv_sn
+                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + (long long)(key_ok ? key : 0) * a.dk_sn;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t v[32];
@@ -754,9 +767,11 @@ inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap
 
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
   if (d == 64)
-    bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.N, a.scale);
+    bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
+                                                 a.scale);
   else
-    bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.N, a.scale);
+    bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
+                                                  a.scale);
   return cudaGetLastError();
 }
 

@@ -45,20 +45,34 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map of a [BH, N, d] bf16 tensor read in 128-row x 64-column boxes
+// Tensor map of a bf16 [B, H, N, d] tensor with element strides s (d
+// contiguous), addressed as {d, n, h, b} and read in 128-row x 64-column boxes
 // with the 128-byte swizzle; rows past N read as zero.
-int make_tile_map(CUtensorMap* m, const void* base, int BH, int N, int d) {
+int make_tile_map(CUtensorMap* m, const void* base, int B, int H, int N, int d, const fa_strides& s) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cuda_fail(cudaErrorNotSupported);
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2u, (cuuint64_t)N * (cuuint64_t)d * 2u};
-  cuuint32_t box[3] = {64u, 128u, 1u};
-  cuuint32_t estride[3] = {1u, 1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)s.n * 2u, (cuuint64_t)s.h * 2u, (cuuint64_t)s.b * 2u};
+  cuuint32_t box[4] = {64u, 128u, 1u, 1u};
+  cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
   return FA_OK;
+}
+
+fa_strides contiguous_strides(int H, int N, int d) {
+  fa_strides s;
+  s.n = d;
+  s.h = (int64_t)N * d;
+  s.b = (int64_t)H * N * d;
+  return s;
+}
+
+// Strides are usable if every row start stays 16-byte aligned.
+bool strides_ok(const fa_strides& s) {
+  return s.b >= 0 && s.h >= 0 && s.n >= 0 && (s.b * 2) % 16 == 0 && (s.h * 2) % 16 == 0 && (s.n * 2) % 16 == 0;
 }
 
 int* device_error_ptr() {
@@ -164,18 +178,21 @@ int fa_get_device_error(void* stream) {
   return value;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-           float scale, int causal, float dropout_p, uint64_t seed, void* stream) {
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                   int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                   void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
+  for (int t = 0; t < 4; ++t)
+    if (!strides_ok(strides[t])) return FA_ERR_ALIGNMENT;
   CUtensorMap mq, mk, mv;
-  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mq, q, B, H, N, d, strides[0])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B, H, N, d, strides[1])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B, H, N, d, strides[2])) != FA_OK) return rc;
   fa::FwdArgs a;
   a.B = B;
   a.H = H;
@@ -185,6 +202,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
   a.seed = seed;
   a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = strides[3].b;
+  a.o_sh = strides[3].h;
+  a.o_sn = strides[3].n;
   a.lse = lse;
   a.err = device_error_ptr();
   if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
@@ -192,6 +212,13 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? dispatch_fwd<64>(mq, mk, mv, a, causal != 0, dropout, st)
                  : dispatch_fwd<128>(mq, mk, mv, a, causal != 0, dropout, st);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, float dropout_p, uint64_t seed, void* stream) {
+  const fa_strides s = contiguous_strides(H, N, d);
+  const fa_strides all[4] = {s, s, s, s};
+  return fa_fwd_strided(q, k, v, o, lse, all, B, H, N, d, scale, causal, dropout_p, seed, stream);
 }
 
 int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,
@@ -239,25 +266,35 @@ int bwd_setup(int B, int H, int N, int d, float scale, int causal, float dropout
 
 }  // namespace
 
-int fa_bwd_prepare(const void* o, const void* dout, const float* lse, int B, int H, int N, int d, void* workspace,
-                   size_t workspace_bytes, void* stream) {
+namespace {
+
+// Strides of the 8 backward tensors, in the order q, k, v, o, dout, dq, dk, dv.
+int bwd_prepare_impl(const void* o, const void* dout, const float* lse, const fa_strides* s, int B, int H, int N,
+                     int d, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, 1.f, 0, 0.f);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
   if (!o || !dout || !lse) return FA_ERR_INVALID_ARG;
-  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(lse, 4) || !strides_ok(s[3]) || !strides_ok(s[4]))
+    return FA_ERR_ALIGNMENT;
   fa::BwdArgs a;
   if ((rc = bwd_setup(B, H, N, d, 1.f, 0, 0.f, 0, workspace, workspace_bytes, &a)) != FA_OK) return rc;
   a.o = static_cast<const __nv_bfloat16*>(o);
+  a.o_sb = s[3].b;
+  a.o_sh = s[3].h;
+  a.o_sn = s[3].n;
   a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.do_sb = s[4].b;
+  a.do_sh = s[4].h;
+  a.do_sn = s[4].n;
   a.lse = lse;
   cudaError_t e = fa::launch_bwd_prepare(a, d, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
-int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
-                     int N, int d, float scale, int causal, float dropout_p, uint64_t seed, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+int bwd_recompute_impl(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                       const fa_strides* s, int B, int H, int N, int d, float scale, int causal, float dropout_p,
+                       uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -265,50 +302,105 @@ int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* do
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dk, 16) ||
       !aligned(dv, 16))
     return FA_ERR_ALIGNMENT;
+  for (int t : {0, 1, 2, 4, 6, 7})
+    if (!strides_ok(s[t])) return FA_ERR_ALIGNMENT;
   fa::BwdArgs a;
   if ((rc = bwd_setup(B, H, N, d, scale, causal, dropout_p, seed, workspace, workspace_bytes, &a)) != FA_OK)
     return rc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dk_sb = s[6].b;
+  a.dk_sh = s[6].h;
+  a.dk_sn = s[6].n;
   a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dv_sb = s[7].b;
+  a.dv_sh = s[7].h;
+  a.dv_sn = s[7].n;
   CUtensorMap mq, mk, mv, mdo;
-  if ((rc = make_tile_map(&mq, q, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mk, k, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mv, v, B * H, N, d)) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mdo, dout, B * H, N, d)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mq, q, B, H, N, d, s[0])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B, H, N, d, s[1])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B, H, N, d, s[2])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mdo, dout, B, H, N, d, s[4])) != FA_OK) return rc;
   cudaError_t e = fa::launch_bwd_recompute(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
-int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+int bwd_finalize_impl(void* dq, const fa_strides* s, int B, int H, int N, int d, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, scale, 0, 0.f);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
   if (!dq) return FA_ERR_INVALID_ARG;
-  if (!aligned(dq, 16)) return FA_ERR_ALIGNMENT;
+  if (!aligned(dq, 16) || !strides_ok(s[5])) return FA_ERR_ALIGNMENT;
   fa::BwdArgs a;
   if ((rc = bwd_setup(B, H, N, d, scale, 0, 0.f, 0, workspace, workspace_bytes, &a)) != FA_OK) return rc;
   a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dq_sb = s[5].b;
+  a.dq_sh = s[5].h;
+  a.dq_sn = s[5].n;
   cudaError_t e = fa::launch_bwd_finalize(a, d, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+void contiguous8(int H, int N, int d, fa_strides* s) {
+  const fa_strides c = contiguous_strides(H, N, d);
+  for (int t = 0; t < 8; ++t) s[t] = c;
+}
+
+}  // namespace
+
+int fa_bwd_prepare(const void* o, const void* dout, const float* lse, int B, int H, int N, int d, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  fa_strides s[8];
+  contiguous8(H, N, d, s);
+  return bwd_prepare_impl(o, dout, lse, s, B, H, N, d, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
+                     int N, int d, float scale, int causal, float dropout_p, uint64_t seed, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  fa_strides s[8];
+  contiguous8(H, N, d, s);
+  return bwd_recompute_impl(q, k, v, dout, dk, dv, s, B, H, N, d, scale, causal, dropout_p, seed, workspace,
+                            workspace_bytes, stream);
+}
+
+int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  fa_strides s[8];
+  contiguous8(H, N, d, s);
+  return bwd_finalize_impl(dq, s, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d, float scale,
+                   int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !strides) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  for (int t = 0; t < 8; ++t)
+    if (!strides_ok(strides[t])) return FA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(B * H, N, d)) return FA_ERR_WORKSPACE;
+  if ((rc = bwd_prepare_impl(o, dout, lse, strides, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK)
+    return rc;
+  if ((rc = bwd_recompute_impl(q, k, v, dout, dk, dv, strides, B, H, N, d, scale, causal, dropout_p, seed, workspace,
+                               workspace_bytes, stream)) != FA_OK)
+    return rc;
+  return bwd_finalize_impl(dq, strides, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
            void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
            void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
-  if (rc == 1) return FA_OK;
-  if (rc != FA_OK) return rc;
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
-    return FA_ERR_ALIGNMENT;
-  if ((rc = fa_bwd_prepare(o, dout, lse, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK) return rc;
-  if ((rc = fa_bwd_recompute(q, k, v, dout, dk, dv, B, H, N, d, scale, causal, dropout_p, seed, workspace,
-                             workspace_bytes, stream)) != FA_OK)
-    return rc;
-  return fa_bwd_finalize(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  fa_strides s[8];
+  contiguous8(H, N, d, s);
+  return fa_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, s, B, H, N, d, scale, causal, dropout_p, seed, workspace,
+                        workspace_bytes, stream);
 }
 
 }  // extern "C"

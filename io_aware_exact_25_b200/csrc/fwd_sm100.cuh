@@ -40,8 +40,9 @@ struct FwdArgs {
   uint32_t drop_threshold;  // keep iff hash32 >= threshold
   float drop_scale;         // 1 / (1 - p)
   uint64_t seed;
-  __nv_bfloat16* o;  // [B,H,N,D]
-  float* lse;        // [B,H,N], natural log
+  __nv_bfloat16* o;            // [B,H,N,D] with element strides o_sb, o_sh, o_sn
+  long long o_sb, o_sh, o_sn;
+  float* lse;                  // [B,H,N] contiguous, natural log
   int* err;          // device error word (may be null)
 };
 
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(320, 1)
   const int tile_rev = blockIdx.x / BH;
   const int bh = blockIdx.x - tile_rev * BH;
   const int cta_tile = CAUSAL ? (n_cta_tiles - 1 - tile_rev) : tile_rev;
+  const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
   const int n_kv_all = (a.N + 127) >> 7;
   const int qt0 = 2 * cta_tile;
   const bool act1 = (qt0 + 1) * 128 < a.N;
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(320, 1)
         if (t == 1 && !act1) break;
         mbar_arrive_expect_tx(&bar_q[t], L::kTile);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, (qt0 + t) * 128, bh,
+          tma_load_4d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, (qt0 + t) * 128, hh, bb,
                       &bar_q[t], pol_once);
       }
       int stage = 0;
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, j * 128, bh,
+            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, j * 128, hh, bb,
                         &bar_kv_full[stage], pol_keep);
           ++issued;
           if (++stage == L::kStages) {
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(320, 1)
       float m_used = -INFINITY;  // running maximum (base-2 units) the P values are taken against
       float l = 0.f;             // running sum of undropped P
       uint32_t rkey = 0;
-      if (DROPOUT) rkey = dropout_row_key(a.seed, (uint32_t)(bh / a.H), (uint32_t)(bh % a.H), (uint32_t)q_row);
+      if (DROPOUT) rkey = dropout_row_key(a.seed, (uint32_t)bb, (uint32_t)hh, (uint32_t)q_row);
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
         if (!mbar_wait(&bar_s[t], j & 1, ab)) {
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool in_range = q_row < a.N;
-        __nv_bfloat16* orow = a.o + ((size_t)bh * a.N + (size_t)(in_range ? q_row : 0)) * D;
+        __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)(in_range ? q_row : 0) * a.o_sn;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t o[32];

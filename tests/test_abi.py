@@ -80,6 +80,19 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
     assert _bwd(lib, p=1.5) == binding.FA_ERR_INVALID_ARG
 
 
+def test_strided_entry_points_check_strides(lib):
+    S = binding.FaStrides
+    good = (S * 8)(*[S(3 * 128 * 64, 128 * 64, 64)] * 8)
+    bad = (S * 8)(*[S(3 * 128 * 64, 128 * 64, 63)] * 8)  # 126-byte rows: misaligned
+    args = (1, 3, 128, 64, 0.125, 0, 0.0, 0)
+    assert lib.fa_fwd_strided(16, 16, 16, 16, 16, bad, *args, None) == binding.FA_ERR_ALIGNMENT
+    assert lib.fa_fwd_strided(16, 16, 16, 16, 16, None, *args, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_strided(16, 16, 16, 16, 16, 16, 16, 16, 16, bad, *args, 16, 1 << 30, None) \
+        == binding.FA_ERR_ALIGNMENT
+    assert lib.fa_bwd_strided(16, 16, 16, 16, 16, 16, 16, 16, 16, good, *args, None, 0, None) \
+        == binding.FA_ERR_WORKSPACE
+
+
 def test_empty_problems_are_noops(lib):
     # nothing to do: success without touching the (absent) device or pointers
     assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == binding.FA_OK
