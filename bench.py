@@ -234,9 +234,17 @@ def run_ours(args, w):
         if rc != 0:
             raise RuntimeError(f"{what}: {binding.strerror(rc)}")
 
+    splits = args.splitkv if args.splitkv > 0 else (lib.fa_splitkv_suggest(B, H, N, d) if args.splitkv < 0 else 1)
+    split_ws_bytes = int(lib.fa_fwd_splitkv_workspace_size(B, H, N, d, splits)) if splits > 1 else 0
+    split_ws = torch.empty(max(split_ws_bytes, 16), dtype=torch.uint8, device=dev)
+
     def fwd():
-        check(lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, w.scale, causal, w.p_drop, w.seed, s),
-              "fa_fwd")
+        if splits > 1:
+            check(lib.fa_fwd_splitkv(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, w.scale, causal, w.p_drop, w.seed,
+                                     splits, P(split_ws), split_ws_bytes, s), "fa_fwd_splitkv")
+        else:
+            check(lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, w.scale, causal, w.p_drop, w.seed, s),
+                  "fa_fwd")
 
     def bwd_prepare():
         check(lib.fa_bwd_prepare(P(o), P(do), P(lse), B, H, N, d, P(work), wsb, s), "fa_bwd_prepare")
@@ -291,7 +299,9 @@ def run_ours(args, w):
 
     if args.no_extras:
         if rank == 0:
-            print(json.dumps({"profiling_run": True, "ms_per_step": elapsed_ms / args.steps,
+            print(json.dumps({"profiling_run": True, "workload": w.name, "splitkv": splits,
+                              "fwd_tflops": w.fwd_flops() / (per_stage_ms[0] * 1e-3) / 1e12,
+                              "ms_per_step": elapsed_ms / args.steps,
                               "stage_ms": dict(zip([n for n, _ in stages], per_stage_ms))}), flush=True)
         if ws > 1:
             dist.destroy_process_group()
@@ -387,7 +397,8 @@ def run_ours(args, w):
             "e2e": {"value": ws * (ff + fb) * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "api": "binding.fwd/binding.bwd (C ABI) with pinned host buffers"},
-            "gpu_launches": args.steps * len(stages),
+            "gpu_launches": args.steps * (len(stages) + (1 if splits > 1 else 0)),
+            "splitkv": splits,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -406,6 +417,8 @@ def main():
     ap.add_argument("--workload", default="long8k_causal")
     ap.add_argument("--cpu-rows", type=int, default=8192,
                     help="causal prefix length of the oracle baseline sample")
+    ap.add_argument("--splitkv", type=int, default=0,
+                    help="forward with fa_fwd_splitkv: number of splits (-1: suggested, 0: plain kernel)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end and CPU-baseline legs (profiling runs)")
     ap.add_argument("--ref-rows", type=int, default=1024,

@@ -91,6 +91,30 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
                    void* stream);
 
 /*
+ * Split-KV forward for problems with few query tiles (small B*H*N leaves
+ * SMs idle: "FlashAttention for Efficient Training" section 6.1, Limited
+ * Parallelism for Small Batch Sizes).  Each query tile's key range is cut
+ * into num_splits consecutive pieces processed by separate CTAs; each piece
+ * writes its normalised partial output O_s (fp32) and logsumexp lse_s, and a
+ * combine pass forms lse = ln sum_s exp(lse_s) and O = sum_s exp(lse_s - lse)
+ * O_s -- the exact merge of softmax pieces over disjoint key sets.  Output,
+ * arguments and errors are those of fa_fwd, plus num_splits in [1, 64]
+ * (1 = the plain kernel) and a caller-owned workspace of at least
+ * fa_fwd_splitkv_workspace_size bytes (16-byte aligned; FA_ERR_WORKSPACE
+ * if too small).  Two launches on `stream`.
+ */
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, float dropout_p, uint64_t seed, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Workspace bytes for fa_fwd_splitkv (0 when num_splits == 1 or invalid). */
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits);
+
+/* A split count for this shape: 1 when the plain grid fills at least half of
+ * the SMs, else as many pieces as fill one wave (at most 16). */
+int fa_splitkv_suggest(int B, int H, int N, int d);
+
+/*
  * Bytes of device workspace fa_bwd needs for this shape: an fp32 dQ
  * accumulator [B,H,N,d] plus two fp32 row vectors (scaled lse and
  * D_i = dO_i . O_i) padded to a multiple of 128 rows.  Returns 0 for an empty

@@ -27,7 +27,8 @@ FA_ERR_CUDA = -5
 FA_ERR_DEVICE = -6
 FA_ERR_TOO_LARGE = -7
 
-EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
+EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
+           "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -60,6 +61,11 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         vp, I, F, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
+        lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, vp, SZ, vp]
+        lib.fa_fwd_splitkv_workspace_size.argtypes = [I, I, I, I, I]
+        lib.fa_fwd_splitkv_workspace_size.restype = SZ
+        lib.fa_splitkv_suggest.argtypes = [I, I, I, I]
+        lib.fa_splitkv_suggest.restype = I
         SP = ctypes.POINTER(FaStrides)
         lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp]
         lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, SZ,
@@ -75,7 +81,7 @@ def load() -> ctypes.CDLL:
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
-        for fn in (lib.fa_fwd, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
+        for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
                    lib.fa_bwd_finalize, lib.fa_bwd_noalloc, lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
@@ -143,6 +149,32 @@ def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=No
     rc = load().fa_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _strides(q, k, v, o), B, H, N, d,
                                float(scale), int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
     _call(rc, "fa_fwd")
+    return o, lse
+
+
+def fwd_splitkv(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, num_splits=None, o=None, lse=None,
+                workspace=None, stream=None):
+    """O and lse via ``fa_fwd_splitkv`` (dense [B,H,N,d] tensors).  The split
+    count defaults to ``fa_splitkv_suggest``."""
+    _check_inputs(q, k, v)
+    _check_dense(q, k, v)
+    B, H, N, d = q.shape
+    lib = load()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        num_splits = int(lib.fa_splitkv_suggest(B, H, N, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    need = int(lib.fa_fwd_splitkv_workspace_size(B, H, N, d, int(num_splits)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                            int(bool(causal)), float(dropout_p), int(seed), int(num_splits), _ptr(workspace),
+                            int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _call(rc, "fa_fwd_splitkv")
     return o, lse
 
 

@@ -107,26 +107,38 @@ uint32_t keep_threshold(float p) {
   return (uint32_t)t;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPLIT>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                cudaStream_t st) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT>;
+  auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT, SPLIT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
   if (e != cudaSuccess) return cuda_fail(e);
-  const long long grid = (long long)a.B * a.H * ((a.N + 255) / 256);
+  const long long grid = (long long)a.B * a.H * ((a.N + 255) / 256) * (SPLIT ? a.num_splits : 1);
   kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  if (SPLIT) {
+    fa::splitkv_combine_kernel<D><<<148 * 8, 256, 0, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return FA_OK;
 }
 
-template <int D>
+template <int D, bool SPLIT>
 int dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                  bool causal, bool dropout, cudaStream_t st) {
   if (causal)
-    return dropout ? launch_fwd<D, true, true>(mq, mk, mv, a, st) : launch_fwd<D, true, false>(mq, mk, mv, a, st);
-  return dropout ? launch_fwd<D, false, true>(mq, mk, mv, a, st) : launch_fwd<D, false, false>(mq, mk, mv, a, st);
+    return dropout ? launch_fwd<D, true, true, SPLIT>(mq, mk, mv, a, st)
+                   : launch_fwd<D, true, false, SPLIT>(mq, mk, mv, a, st);
+  return dropout ? launch_fwd<D, false, true, SPLIT>(mq, mk, mv, a, st)
+                 : launch_fwd<D, false, false, SPLIT>(mq, mk, mv, a, st);
+}
+
+size_t splitkv_bytes(int B, int H, int N, int d, int splits) {
+  const size_t rows = (size_t)B * H * N * (size_t)splits;
+  return fa::round_up(rows * d * 4, 256) + fa::round_up(rows * 4, 256);
 }
 
 __global__ void dropout_mask_kernel(int H, int N, uint32_t threshold, uint64_t seed, const int32_t* heads,
@@ -178,9 +190,11 @@ int fa_get_device_error(void* stream) {
   return value;
 }
 
-int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
-                   int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
-                   void* stream) {
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides, int B,
+             int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int num_splits,
+             void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -189,6 +203,10 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
     return FA_ERR_ALIGNMENT;
   for (int t = 0; t < 4; ++t)
     if (!strides_ok(strides[t])) return FA_ERR_ALIGNMENT;
+  if (num_splits > 1) {
+    if (!workspace || workspace_bytes < splitkv_bytes(B, H, N, d, num_splits)) return FA_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
+  }
   CUtensorMap mq, mk, mv;
   if ((rc = make_tile_map(&mq, q, B, H, N, d, strides[0])) != FA_OK) return rc;
   if ((rc = make_tile_map(&mk, k, B, H, N, d, strides[1])) != FA_OK) return rc;
@@ -206,12 +224,60 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
   a.o_sh = strides[3].h;
   a.o_sn = strides[3].n;
   a.lse = lse;
+  a.num_splits = num_splits;
+  a.part_o = nullptr;
+  a.part_lse = nullptr;
+  if (num_splits > 1) {
+    a.part_o = static_cast<float*>(workspace);
+    a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          fa::round_up((size_t)B * H * N * (size_t)num_splits * d * 4, 256));
+  }
   a.err = device_error_ptr();
   if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
   const bool dropout = dropout_p > 0.f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? dispatch_fwd<64>(mq, mk, mv, a, causal != 0, dropout, st)
-                 : dispatch_fwd<128>(mq, mk, mv, a, causal != 0, dropout, st);
+  if (num_splits > 1)
+    return d == 64 ? dispatch_fwd<64, true>(mq, mk, mv, a, causal != 0, dropout, st)
+                   : dispatch_fwd<128, true>(mq, mk, mv, a, causal != 0, dropout, st);
+  return d == 64 ? dispatch_fwd<64, false>(mq, mk, mv, a, causal != 0, dropout, st)
+                 : dispatch_fwd<128, false>(mq, mk, mv, a, causal != 0, dropout, st);
+}
+
+}  // namespace
+
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                   int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                   void* stream) {
+  return fwd_impl(q, k, v, o, lse, strides, B, H, N, d, scale, causal, dropout_p, seed, 1, nullptr, 0, stream);
+}
+
+int fa_splitkv_suggest(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.f, 0, 0.f) != FA_OK) return 1;
+  // Split only when the plain grid leaves more than half of the 148 SMs idle,
+  // and then into as many pieces as fill one wave (partials cost an extra
+  // write, read and combine pass, and a second, ragged wave costs more).
+  const long long ctas = (long long)B * H * ((N + 255) / 256);
+  const int nkv = (N + 127) / 128;
+  if (2 * ctas > 148) return 1;
+  long long s = 148 / ctas;
+  if (s > nkv / 2) s = nkv / 2;  // at least two key tiles per split
+  if (s > 16) s = 16;
+  return s < 1 ? 1 : (int)s;
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
+  if (check_common(B, H, N, d, 1.f, 0, 0.f) != FA_OK || num_splits < 1 || num_splits > 64) return 0;
+  return num_splits > 1 ? splitkv_bytes(B, H, N, d, num_splits) : 0;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, float dropout_p, uint64_t seed, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (num_splits < 1 || num_splits > 64) return FA_ERR_INVALID_ARG;
+  const fa_strides s = contiguous_strides(H, N, d);
+  const fa_strides all[4] = {s, s, s, s};
+  return fwd_impl(q, k, v, o, lse, all, B, H, N, d, scale, causal, dropout_p, seed, num_splits, workspace,
+                  workspace_bytes, stream);
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,

@@ -44,6 +44,12 @@ struct FwdArgs {
   long long o_sb, o_sh, o_sn;
   float* lse;                  // [B,H,N] contiguous, natural log
   int* err;          // device error word (may be null)
+  // split-KV (SPLIT kernels only): each CTA covers key tiles [j0, j1) of its
+  // query tiles, split = blockIdx % num_splits, and writes O / l (fp32) and
+  // its lse into part_o [split][BH][N][D] and part_lse [split][BH][N]
+  int num_splits;
+  float* part_o;
+  float* part_lse;
 };
 
 // Of every 8 pairs of probabilities, this many take the exponential on the
@@ -64,7 +70,7 @@ struct FwdLayout {
   static constexpr uint32_t kColO = 256;  // O_t at kColO + D * t
 };
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPLIT>
 __global__ void __launch_bounds__(320, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -95,15 +101,29 @@ __global__ void __launch_bounds__(320, 1)
   // near lockstep, so the K/V tiles they read stay in L2.
   const int BH = a.B * a.H;
   const int n_cta_tiles = (a.N + 255) >> 8;
-  const int tile_rev = blockIdx.x / BH;
-  const int bh = blockIdx.x - tile_rev * BH;
+  const int split = SPLIT ? (int)(blockIdx.x % (unsigned)a.num_splits) : 0;
+  const int work = SPLIT ? (int)(blockIdx.x / (unsigned)a.num_splits) : (int)blockIdx.x;
+  const int tile_rev = work / BH;
+  const int bh = work - tile_rev * BH;
   const int cta_tile = CAUSAL ? (n_cta_tiles - 1 - tile_rev) : tile_rev;
   const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
   const int n_kv_all = (a.N + 127) >> 7;
   const int qt0 = 2 * cta_tile;
   const bool act1 = (qt0 + 1) * 128 < a.N;
-  const int nkv0 = CAUSAL ? qt0 + 1 : n_kv_all;
-  const int nkv1 = act1 ? (CAUSAL ? qt0 + 2 : n_kv_all) : 0;
+  // key tiles each Q tile sees: [0, end_t)
+  const int end0 = CAUSAL ? qt0 + 1 : n_kv_all;
+  const int end1 = act1 ? (CAUSAL ? qt0 + 2 : n_kv_all) : 0;
+  const int end_max = end0 > end1 ? end0 : end1;
+  // this CTA's share [j0, j0 + span) of that range; nkv_t counts the tiles
+  // tile t processes here, local index jj = j - j0 drives the pipelines
+  int j0 = 0, span = end_max;
+  if (SPLIT) {
+    const int chunk = (end_max + a.num_splits - 1) / a.num_splits;
+    j0 = split * chunk;
+    span = max(0, min(end_max, j0 + chunk) - j0);
+  }
+  const int nkv0 = max(0, min(end0, j0 + span) - j0);
+  const int nkv1 = max(0, min(end1, j0 + span) - j0);
   const int nkv_max = nkv0 > nkv1 ? nkv0 : nkv1;
 
   if (threadIdx.x == 0) {
@@ -164,7 +184,7 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, j * 128, hh, bb,
+            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, (j0 + j) * 128, hh, bb,
                         &bar_kv_full[stage], pol_keep);
           ++issued;
           if (++stage == L::kStages) {
@@ -220,10 +240,12 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(&bar_pv[t]);
         return true;
       };
-      if (ok && mbar_wait(&bar_kv_full[0], 0, ab)) {
+      if (nkv_max == 0) {
+        ok = false;  // nothing to do in this split
+      } else if (ok && mbar_wait(&bar_kv_full[0], 0, ab)) {
         tc_fence_after();
         const uint32_t sK0 = sbase + L::kOffKV;
-        issue_s(0, sK0);
+        if (nkv0 > 0) issue_s(0, sK0);
         if (nkv1 > 0) issue_s(1, sK0);
         mma_commit(&bar_kv_empty[0]);
       } else {
@@ -297,12 +319,12 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
-        const bool last = j == nkv - 1;
-        // key 128 j + c is visible to query 128 (qt0 + t) + r iff c < lim;
+        const int jg = j0 + j;  // global key tile
+        // key 128 jg + c is visible to query 128 (qt0 + t) + r iff c < lim;
         // only the diagonal tile (causal) or the ragged last tile masks
         int lim = 128;
-        if (CAUSAL && last) lim = r + 1;
-        if (!CAUSAL && last && (a.N & 127)) lim = a.N - j * 128;
+        if (CAUSAL && jg == qt0 + t) lim = r + 1;
+        if (!CAUSAL && jg == n_kv_all - 1 && (a.N & 127)) lim = a.N - jg * 128;
         if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -373,7 +395,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
           if (DROPOUT) {
-            const uint32_t col = (uint32_t)(j * 128 + 2 * c);
+            const uint32_t col = (uint32_t)(jg * 128 + 2 * c);
             p0 = dropout_hash(rkey, col) >= a.drop_threshold ? p0 * a.drop_scale : 0.f;
             p1 = dropout_hash(rkey, col + 1) >= a.drop_threshold ? p1 * a.drop_scale : 0.f;
           }
@@ -402,26 +424,52 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(&bar_p[t]);
       }
       // epilogue: O = O_t / l, lse = (m + log2 l) ln 2
-      if (ok && mbar_wait(&bar_pv[t], (nkv - 1) & 1, ab)) {
+      const bool in_range = q_row < a.N;
+      if (SPLIT && nkv == 0) {
+        // this split holds no key tile of this query tile: an empty partial
+        if (in_range && ok) {
+          float* prow = a.part_o + (((size_t)split * BH + bh) * a.N + q_row) * D;
+#pragma unroll
+          for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(prow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          a.part_lse[((size_t)split * BH + bh) * a.N + q_row] = -INFINITY;
+        }
+      } else if (ok && mbar_wait(&bar_pv[t], (nkv - 1) & 1, ab)) {
         tc_fence_after();
         const float inv_l = 1.f / l;
-        const bool in_range = q_row < a.N;
-        __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)(in_range ? q_row : 0) * a.o_sn;
+        const float lse_row = (m_used + log2f(l)) * 0.69314718055994531f;
+        if (SPLIT) {
+          float* prow = a.part_o + (((size_t)split * BH + bh) * a.N + (size_t)(in_range ? q_row : 0)) * D;
 #pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
-          uint32_t o[32];
-          tmem_ld32_sync(tO + 32u * c4, o);
-          uint32_t w[16];
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_ld32_sync(tO + 32u * c4, o);
+            if (in_range) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            w[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
-          if (in_range) {
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              st_global_v4(orow + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+              for (int v4 = 0; v4 < 8; ++v4)
+                *reinterpret_cast<float4*>(prow + 32 * c4 + 4 * v4) =
+                    make_float4(__uint_as_float(o[4 * v4]) * inv_l, __uint_as_float(o[4 * v4 + 1]) * inv_l,
+                                __uint_as_float(o[4 * v4 + 2]) * inv_l, __uint_as_float(o[4 * v4 + 3]) * inv_l);
+            }
           }
+          if (in_range) a.part_lse[((size_t)split * BH + bh) * a.N + q_row] = lse_row;
+        } else {
+          __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)(in_range ? q_row : 0) * a.o_sn;
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_ld32_sync(tO + 32u * c4, o);
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              w[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+            if (in_range) {
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4)
+                st_global_v4(orow + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+            }
+          }
+          if (in_range) a.lse[(size_t)bh * a.N + q_row] = lse_row;
         }
-        if (in_range) a.lse[(size_t)bh * a.N + q_row] = (m_used + log2f(l)) * 0.69314718055994531f;
       }
     }
   }
@@ -431,6 +479,42 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge the split-KV partials of one row: lse = ln sum_s exp(lse_s) and
+// O = sum_s exp(lse_s - lse) O_s, the exact combination of softmax pieces over
+// disjoint key ranges.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) splitkv_combine_kernel(const FwdArgs a) {
+  constexpr int kPer = D / 32;
+  const int BH = a.B * a.H;
+  const long long rows = (long long)BH * a.N;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r = warp0; r < rows; r += nwarps) {
+    float mx = -INFINITY;
+    for (int s = 0; s < a.num_splits; ++s) mx = fmaxf(mx, a.part_lse[(size_t)s * rows + r]);
+    float acc[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+    float wsum = 0.f;
+    for (int s = 0; s < a.num_splits; ++s) {
+      const float ls = a.part_lse[(size_t)s * rows + r];
+      const float w = (ls == -INFINITY) ? 0.f : __expf(ls - mx);
+      wsum += w;
+      const float* src = a.part_o + ((size_t)s * rows + r) * D + lane * kPer;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+    }
+    const float inv = 1.f / wsum;
+    const int bh = (int)(r / a.N), i = (int)(r - (long long)bh * a.N);
+    const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+    __nv_bfloat16* orow = a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+    if (lane == 0) a.lse[r] = mx + logf(wsum);
   }
 }
 

@@ -60,6 +60,8 @@ WORKLOADS = {
     "long8k_causal": Workload("long8k_causal", 2, 16, 8192, 128, True, 0.0, 2, qkv_scale=0.5),
     "long32k_causal": Workload("long32k_causal", 1, 16, 32768, 128, True, 0.0, 3, offset_norm=2.0),
     "long64k_causal_dropout": Workload("long64k_causal_dropout", 1, 8, 65536, 128, True, 0.1, 4),
+    # few query tiles (64 CTAs of work for 148 SMs): the split-KV case
+    "smallbatch16k": Workload("smallbatch16k", 1, 1, 16384, 128, False, 0.0, 5),
 }
 
 

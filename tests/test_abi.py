@@ -93,6 +93,24 @@ def test_strided_entry_points_check_strides(lib):
         == binding.FA_ERR_WORKSPACE
 
 
+def test_splitkv_workspace_and_arguments(lib):
+    B, H, N, d = 1, 2, 1000, 128
+    rows = B * H * N * 3
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, N, d, 3) == up(rows * d * 4) + up(rows * 4)
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, N, d, 1) == 0
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, N, d, 65) == 0
+    args = (B, H, N, d, 0.1, 0, 0.0, 0)
+    assert lib.fa_fwd_splitkv(16, 16, 16, 16, 16, *args, 0, 16, 1 << 30, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_splitkv(16, 16, 16, 16, 16, *args, 3, None, 0, None) == binding.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_splitkv(16, 16, 16, 16, 16, *args, 3, 16, 100, None) == binding.FA_ERR_WORKSPACE
+    assert lib.fa_splitkv_suggest(2, 16, 8192, 128) == 1       # 512 CTAs fill the GPU
+    assert lib.fa_splitkv_suggest(1, 2, 16384, 128) == 1       # 128 CTAs: more than half full
+    assert lib.fa_splitkv_suggest(1, 1, 16384, 128) == 2       # 64 CTAs -> one wave of 128
+
+
 def test_empty_problems_are_noops(lib):
     # nothing to do: success without touching the (absent) device or pointers
     assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == binding.FA_OK
