@@ -75,6 +75,8 @@ def _load():
         lib.orc_hash_constant.restype = ctypes.c_uint32
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = ctypes.c_int
+        lib.orc_set_block_mask.argtypes = [u8p, I, I]
+        lib.orc_set_block_mask.restype = None
         _lib = lib
         return lib
 
@@ -121,16 +123,51 @@ def _p(a, ctype):
     return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctype))
 
 
+class _BlockMask:
+    """Installs a block mask for the oracle calls made inside the ``with``.
+
+    ``mask`` is ``[heads, nt, nt]`` with heads 1 (shared by every head) or H
+    and ``nt = ceil(N / tile)``; a zero at ``[h, a, c]`` hides keys of tile c
+    from queries of tile a.  The C side keeps the pointer per thread, so the
+    array is held here until the call returns.
+    """
+
+    def __init__(self, mask, H, N, tile):
+        self.arr = None
+        if mask is None:
+            return
+        if not isinstance(mask, np.ndarray):
+            mask = mask.detach().to("cpu").numpy()
+        a = np.ascontiguousarray(np.asarray(mask) != 0, dtype=np.uint8)
+        nt = (N + tile - 1) // tile
+        if a.ndim != 3 or a.shape[0] not in (1, H) or a.shape[1:] != (nt, nt):
+            raise ValueError(f"block mask must be [1 or H, {nt}, {nt}], got {a.shape}")
+        self.arr, self.tile = a, int(tile)
+
+    def __enter__(self):
+        if self.arr is not None:
+            _load().orc_set_block_mask(_p(self.arr, ctypes.c_uint8), self.arr.shape[0], self.tile)
+        return self
+
+    def __exit__(self, *exc):
+        if self.arr is not None:
+            _load().orc_set_block_mask(None, 1, 128)
+        return False
+
+
 def num_threads() -> int:
     """OpenMP threads the oracle uses (``OMP_NUM_THREADS`` or all cores)."""
     return int(_load().orc_num_threads())
 
 
-def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None):
+def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None,
+            block_mask=None, block=128):
     """O_i and lse_i for the selected heads (bh = b*H + h) and query rows.
 
     Returns ``(o, lse)`` as float64 arrays of shape ``[nheads, nrows, d]`` and
-    ``[nheads, nrows]``.
+    ``[nheads, nrows]``.  ``block_mask`` (``[1 or H, nt, nt]`` over
+    ``block``-sized tiles) hides whole key tiles; a row that sees no key gets
+    O = 0 and lse = -inf.
     """
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     f64 = _kind(qb, kb, vb)
@@ -139,16 +176,18 @@ def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=N
     rs, nr = _idx(rows, N)
     o = np.empty((nh, nr, d), np.float64)
     lse = np.empty((nh, nr), np.float64)
-    rc = _load().orc_forward(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, f64,
-                             B, H, N, d, float(scale), int(bool(causal)), float(p_drop), int(seed),
-                             _p(hs, ctypes.c_int32), nh, _p(rs, ctypes.c_int32), nr,
-                             _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
+    with _BlockMask(block_mask, H, N, block):
+        rc = _load().orc_forward(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, f64,
+                                 B, H, N, d, float(scale), int(bool(causal)), float(p_drop), int(seed),
+                                 _p(hs, ctypes.c_int32), nh, _p(rs, ctypes.c_int32), nr,
+                                 _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
     if rc:
         raise RuntimeError(f"orc_forward failed ({rc})")
     return o, lse
 
 
-def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None):
+def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None,
+               block_mask=None, block=128):
     """dQ_i and D_i for the selected query rows.
 
     Returns ``(dq, D, max_rel_dev)``; ``max_rel_dev`` is the largest relative
@@ -163,17 +202,19 @@ def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=Non
     dq = np.empty((nh, nr, d), np.float64)
     D = np.empty((nh, nr), np.float64)
     dev = ctypes.c_double(0.0)
-    rc = _load().orc_backward_q(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
-                                db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
-                                float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,
-                                _p(rs, ctypes.c_int32), nr, _p(dq, ctypes.c_double),
-                                _p(D, ctypes.c_double), ctypes.byref(dev))
+    with _BlockMask(block_mask, H, N, block):
+        rc = _load().orc_backward_q(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+                                    db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
+                                    float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,
+                                    _p(rs, ctypes.c_int32), nr, _p(dq, ctypes.c_double),
+                                    _p(D, ctypes.c_double), ctypes.byref(dev))
     if rc:
         raise RuntimeError(f"orc_backward_q failed ({rc})")
     return dq, D, dev.value
 
 
-def backward_kv(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, keys=None):
+def backward_kv(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, keys=None,
+                block_mask=None, block=128):
     """dK_j and dV_j for the selected heads and key rows.
 
     Returns ``(dk, dv)`` of shape ``[nheads, nkeys, d]``.
@@ -185,11 +226,12 @@ def backward_kv(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=No
     ks, nk = _idx(keys, N)
     dk = np.empty((nh, nk, d), np.float64)
     dv = np.empty((nh, nk, d), np.float64)
-    rc = _load().orc_backward_kv(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
-                                 db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
-                                 float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,
-                                 _p(ks, ctypes.c_int32), nk, _p(dk, ctypes.c_double),
-                                 _p(dv, ctypes.c_double))
+    with _BlockMask(block_mask, H, N, block):
+        rc = _load().orc_backward_kv(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+                                     db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
+                                     float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,
+                                     _p(ks, ctypes.c_int32), nk, _p(dk, ctypes.c_double),
+                                     _p(dv, ctypes.c_double))
     if rc:
         raise RuntimeError(f"orc_backward_kv failed ({rc})")
     return dk, dv

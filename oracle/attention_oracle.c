@@ -40,7 +40,12 @@
  *  - logsumexp statistic: same page, section 3.2 (log_softmax equation);
  *  - dV = P^T dO: same page, section 3.2 (Integration with Autograd Engines);
  *  - dropout fused after softmax scaling: same page, section 3 (Fused Kernel
- *    Design) and section 6.1 (Kernel Fusion Overhead).
+ *    Design) and section 6.1 (Kernel Fusion Overhead);
+ *  - block-sparse attention, only non-zero blocks of the attention matrix
+ *    computed: same page, section 3.2 (Block-Sparse Attention Support).  An
+ *    optional mask over tile x tile blocks hides keys (s_ij = -inf); a row
+ *    that sees no key at all gets P = 0, O = 0 and lse = -inf (the pages do
+ *    not say; this is the limit of an empty softmax taken as zero weight).
  * The pages print garbled dQ formulas; the dQ/dK expressions here are the
  * chain rule, pinned by finite differences in the tests.
  *
@@ -71,6 +76,10 @@ typedef struct {
     int causal;
     double p_drop;
     uint64_t seed;
+    /* optional block mask: bmask[hm][i / tile][j / tile] == 0 hides keys j from
+     * queries i (hm = 0 if bmask_heads == 1, else the head h) */
+    const uint8_t *bmask;
+    int bmask_heads, bmask_tile;
 } problem_t;
 
 /* A row of one [B,H,N,d] input: base pointer plus its element type. */
@@ -163,12 +172,22 @@ static int keep_elem(const problem_t *pb, int bh, int i, int j) {
 
 /* -------------------------------------------------------- one query row */
 
-/* Scores s_ij for row i of head bh, then the row statistics m_i and l_i. */
+/* Is key j hidden from query i by the block mask? */
+static int block_masked(const problem_t *pb, int bh, int i, int j) {
+    if (!pb->bmask) return 0;
+    const int nt = (pb->N + pb->bmask_tile - 1) / pb->bmask_tile;
+    const int hm = pb->bmask_heads == 1 ? 0 : bh % pb->H;
+    return pb->bmask[((size_t)hm * nt + (size_t)(i / pb->bmask_tile)) * nt + (size_t)(j / pb->bmask_tile)] == 0;
+}
+
+/* Scores s_ij for row i of head bh, then the row statistics m_i and l_i.
+ * A row that sees no key (every key hidden by the block mask) has
+ * m = -inf and l = 0; its probabilities are taken as 0. */
 static void row_scores(const problem_t *pb, int bh, int i, double *s, double *m_out, double *l_out) {
     row_t qi = row_ptr(pb, pb->q, bh, i);
     double m = -INFINITY;
     for (int j = 0; j < pb->N; ++j) {
-        if (pb->causal && j > i) {
+        if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {
             s[j] = -INFINITY;
         } else {
             s[j] = pb->scale * dot_rows(qi, row_ptr(pb, pb->k, bh, j), pb->d);
@@ -176,13 +195,14 @@ static void row_scores(const problem_t *pb, int bh, int i, double *s, double *m_
         if (s[j] > m) m = s[j];
     }
     double l = 0.0;
-    for (int j = 0; j < pb->N; ++j) l += exp(s[j] - m); /* exp(-inf) = 0 */
+    if (m != -INFINITY)
+        for (int j = 0; j < pb->N; ++j) l += exp(s[j] - m); /* exp(-inf) = 0 */
     *m_out = m;
     *l_out = l;
 }
 
-/* P_ij for one score, from the row statistics. */
-static double prob(double s, double m, double l) { return exp(s - m) / l; }
+/* P_ij for one score, from the row statistics (0 for a row with no key). */
+static double prob(double s, double m, double l) { return l > 0.0 ? exp(s - m) / l : 0.0; }
 
 /* O_i (d values) and lse_i for one query row. */
 static void row_forward(const problem_t *pb, int bh, int i, double *s, double *o, double *lse) {
@@ -197,7 +217,7 @@ static void row_forward(const problem_t *pb, int bh, int i, double *s, double *o
         row_t vj = row_ptr(pb, pb->v, bh, j);
         for (int c = 0; c < pb->d; ++c) o[c] += pd * elem(vj, c);
     }
-    *lse = m + log(l);
+    *lse = l > 0.0 ? m + log(l) : -INFINITY;
 }
 
 /*
@@ -255,7 +275,28 @@ static problem_t make_problem(const void *q, const void *k, const void *v, const
     pb.causal = causal;
     pb.p_drop = p_drop;
     pb.seed = seed;
+    pb.bmask = NULL;
+    pb.bmask_heads = 1;
+    pb.bmask_tile = 128;
     return pb;
+}
+
+/* Block mask used by the next orc_forward / orc_backward_q / orc_backward_kv
+ * call of this thread (NULL: none).  mask is [heads][nt][nt] bytes with
+ * nt = ceil(N / tile); heads is 1 (shared) or H. */
+static _Thread_local const uint8_t *tl_bmask = NULL;
+static _Thread_local int tl_bmask_heads = 1, tl_bmask_tile = 128;
+
+void orc_set_block_mask(const uint8_t *mask, int heads, int tile) {
+    tl_bmask = mask;
+    tl_bmask_heads = heads;
+    tl_bmask_tile = tile > 0 ? tile : 128;
+}
+
+static void apply_block_mask(problem_t *pb) {
+    pb->bmask = tl_bmask;
+    pb->bmask_heads = tl_bmask_heads;
+    pb->bmask_tile = tl_bmask_tile;
 }
 
 static int check_args(int B, int H, int N, int d, double p_drop) {
@@ -277,6 +318,7 @@ int orc_forward(const void *q, const void *k, const void *v, int f64, int B, int
     if (check_args(B, H, N, d, p_drop)) return -1;
     init_consts();
     problem_t pb = make_problem(q, k, v, NULL, f64, B, H, N, d, scale, causal, p_drop, seed);
+    apply_block_mask(&pb);
     int nh = heads ? nheads : B * H;
     int nr = rows ? nrows : N;
     int64_t total = (int64_t)nh * nr;
@@ -313,6 +355,7 @@ int orc_backward_q(const void *q, const void *k, const void *v, const void *dout
     if (check_args(B, H, N, d, p_drop)) return -1;
     init_consts();
     problem_t pb = make_problem(q, k, v, dout, f64, B, H, N, d, scale, causal, p_drop, seed);
+    apply_block_mask(&pb);
     int nh = heads ? nheads : B * H;
     int nr = rows ? nrows : N;
     int64_t total = (int64_t)nh * nr;
@@ -359,6 +402,7 @@ int orc_backward_kv(const void *q, const void *k, const void *v, const void *dou
     if (check_args(B, H, N, d, p_drop)) return -1;
     init_consts();
     problem_t pb = make_problem(q, k, v, dout, f64, B, H, N, d, scale, causal, p_drop, seed);
+    apply_block_mask(&pb);
     int nh = heads ? nheads : B * H;
     int nk = keys ? nkeys : N;
     int first_row = 0;
@@ -435,6 +479,7 @@ int orc_backward_kv(const void *q, const void *k, const void *v, const void *dou
         row_t vj = row_ptr(&pb, pb.v, bh, j);
         int i0 = causal ? j : 0;
         for (int i = i0; i < N; ++i) {
+            if (block_masked(&pb, bh, i, j)) continue;
             size_t su = (size_t)hi * nstat + (size_t)(i - first_row);
             row_t qi = row_ptr(&pb, pb.q, bh, i);
             row_t doi = row_ptr(&pb, pb.dout, bh, i);

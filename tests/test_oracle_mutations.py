@@ -16,16 +16,22 @@ SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
 
 MUTANTS = {
     "drop_minus_D_in_dS": ("double ds = p * (dp - D);", "double ds = p * dp;"),
-    "causal_mask_transposed": ("if (pb->causal && j > i) {", "if (pb->causal && j < i) {"),
-    "causal_mask_off_by_one": ("if (pb->causal && j > i) {", "if (pb->causal && j >= i) {"),
-    "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "causal_mask_transposed": ("if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
+                               "if ((pb->causal && j < i) || block_masked(pb, bh, i, j)) {"),
+    "causal_mask_off_by_one": ("if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
+                               "if ((pb->causal && j >= i) || block_masked(pb, bh, i, j)) {"),
+    "lse_without_max": ("*lse = l > 0.0 ? m + log(l) : -INFINITY;", "*lse = l > 0.0 ? log(l) : -INFINITY;"),
     "dropout_scale_inverted": ("const double inv_keep = 1.0 / (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;",
                                "const double inv_keep = (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;"),
     "dq_missing_scale": ("for (int c = 0; c < pb->d; ++c) dq[c] *= pb->scale;", ""),
     "dk_uses_k_not_q": ("dkj[c] += ds * elem(qi, c);", "dkj[c] += ds * elem(kj, c);"),
     "dv_without_dropout_mask": ("double pd = p * z;", "double pd = p;"),
-    "softmax_not_normalised": ("static double prob(double s, double m, double l) { return exp(s - m) / l; }",
-                               "static double prob(double s, double m, double l) { (void)l; return exp(s - m); }"),
+    "softmax_not_normalised": ("return l > 0.0 ? exp(s - m) / l : 0.0;", "return l > 0.0 ? exp(s - m) : 0.0;"),
+    "block_mask_transposed": ("(size_t)(i / pb->bmask_tile)) * nt + (size_t)(j / pb->bmask_tile)]",
+                              "(size_t)(j / pb->bmask_tile)) * nt + (size_t)(i / pb->bmask_tile)]"),
+    "block_mask_head_ignored": ("const int hm = pb->bmask_heads == 1 ? 0 : bh % pb->H;", "const int hm = 0;"),
+    "key_pass_ignores_block_mask": ("if (block_masked(&pb, bh, i, j)) continue;", ""),
+    "empty_row_lse_zero": ("*lse = l > 0.0 ? m + log(l) : -INFINITY;", "*lse = l > 0.0 ? m + log(l) : 0.0;"),
     "hash_constant_typo": ("C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32);",
                            "C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32) + 2u;"),
     "threshold_floor": ("double t = ceil(p * 4294967296.0);", "double t = floor(p * 4294967296.0);"),

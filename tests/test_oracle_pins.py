@@ -338,3 +338,118 @@ def test_pages_memory_arithmetic():
     assert accounting.standard_attention_bandwidth(b["B"], b["N"], b["t_s"]) > b["expect_min_bytes_per_s"]
     c = ref["tile_saving_8192_512"]
     assert accounting.tiling_memory_saving(c["N"], c["tile"]) == c["expect_factor"]
+
+
+# ----------------------------------------------------- block-sparse pins
+# Block-sparse attention ("FlashAttention for Efficient Training", section
+# 3.2, Block-Sparse Attention Support): a 0/1 mask over tile x tile blocks
+# hides whole key blocks.  Small tiles keep these cases tiny.
+
+def _random_block_mask(H, nt, seed, density=0.5, keep_diagonal=True):
+    g = torch.Generator().manual_seed(seed)
+    m = (torch.rand(H, nt, nt, generator=g) < density).to(torch.uint8)
+    if keep_diagonal:
+        m[:, torch.arange(nt), torch.arange(nt)] = 1
+    return m
+
+
+def _dense_mask(bm, N, tile, causal):
+    """Element mask (True = visible) from a block mask, as torch SDPA takes it."""
+    el = bm.to(torch.bool).repeat_interleave(tile, 1).repeat_interleave(tile, 2)[:, :N, :N]
+    if causal:
+        el = el & torch.ones(N, N, dtype=torch.bool).tril()
+    return el
+
+
+@pytest.mark.parametrize("causal,shared", [(False, False), (True, False), (False, True)])
+def test_block_mask_matches_torch_element_mask(causal, shared):
+    B, H, N, d, tile = 2, 3, 44, 8, 8           # 6 tiles, the last one ragged (4 rows)
+    x = make_inputs(B, H, N, d, seed=31)
+    nt = (N + tile - 1) // tile
+    bm = _random_block_mask(1 if shared else H, nt, seed=32)
+    sc = 0.3
+    el = _dense_mask(bm, N, tile, causal).expand(H, N, N).unsqueeze(0)
+    q, k, v = (_f64(x[n]).requires_grad_(True) for n in ("q", "k", "v"))
+    o_ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=el, scale=sc)
+    o_ref.backward(_f64(x["do"]))
+    o, lse = oracle.forward(x["q"], x["k"], x["v"], sc, causal=causal, block_mask=bm, block=tile)
+    assert np.max(np.abs(o - o_ref.detach().reshape(B * H, N, d).numpy())) < 1e-12
+    s = (_f64(x["q"]) @ _f64(x["k"]).transpose(-1, -2)) * sc
+    lse_ref = torch.logsumexp(s.masked_fill(~el, float("-inf")), dim=-1).reshape(B * H, N).numpy()
+    assert np.max(np.abs(lse - lse_ref)) < 1e-12
+    dq, _, dev = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], sc, causal=causal,
+                                   block_mask=bm, block=tile)
+    dk, dv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], sc, causal=causal,
+                                block_mask=bm, block=tile)
+    assert dev < 1e-12
+    for got, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        assert np.max(np.abs(got - ref.reshape(B * H, N, d).numpy())) < 1e-11
+
+
+def test_all_ones_block_mask_is_dense_attention():
+    x = make_inputs(1, 2, 40, 8, seed=33)
+    ones = np.ones((1, 5, 5), np.uint8)
+    for causal in (False, True):
+        a = oracle.forward(x["q"], x["k"], x["v"], 0.3, causal=causal)
+        b = oracle.forward(x["q"], x["k"], x["v"], 0.3, causal=causal, block_mask=ones, block=8)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+        ga = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], 0.3, causal=causal)
+        gb = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], 0.3, causal=causal, block_mask=ones, block=8)
+        assert np.array_equal(ga[0], gb[0]) and np.array_equal(ga[1], gb[1])
+
+
+def test_block_diagonal_mask_is_independent_problems():
+    """With only diagonal blocks, each tile is its own N = tile problem."""
+    B, H, N, d, tile = 1, 2, 32, 8, 8
+    x = make_inputs(B, H, N, d, seed=34)
+    eye = np.eye(N // tile, dtype=np.uint8)[None]
+    o, lse = oracle.forward(x["q"], x["k"], x["v"], 0.4, causal=True, block_mask=eye, block=tile)
+    dq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], 0.4, causal=True,
+                                 block_mask=eye, block=tile)
+    dk, dv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], 0.4, causal=True,
+                                block_mask=eye, block=tile)
+    for a in range(N // tile):
+        sl = slice(a * tile, (a + 1) * tile)
+        sub = {n: x[n][:, :, sl].contiguous() for n in x}
+        o_s, lse_s = oracle.forward(sub["q"], sub["k"], sub["v"], 0.4, causal=True)
+        dq_s, _, _ = oracle.backward_q(sub["q"], sub["k"], sub["v"], sub["do"], 0.4, causal=True)
+        dk_s, dv_s = oracle.backward_kv(sub["q"], sub["k"], sub["v"], sub["do"], 0.4, causal=True)
+        assert np.max(np.abs(lse[:, sl] - lse_s)) < 1e-13
+        for got, ref in ((o, o_s), (dq, dq_s), (dk, dk_s), (dv, dv_s)):
+            assert np.max(np.abs(got[:, sl] - ref)) < 1e-13
+
+
+def test_rows_that_see_no_key():
+    """A query tile whose mask row is all zero: O = 0, lse = -inf, dQ = 0, and
+    its rows add nothing to dK and dV (the other rows match torch run on them
+    alone)."""
+    B, H, N, d, tile = 1, 2, 40, 8, 8
+    x = make_inputs(B, H, N, d, seed=35)
+    bm = np.ones((H, 5, 5), np.uint8)
+    bm[0, 2, :] = 0                               # head 0: rows 16..23 see nothing
+    bm[1, 4, :] = 0                               # head 1: the last tile
+    sc = 0.3
+    o, lse = oracle.forward(x["q"], x["k"], x["v"], sc, block_mask=bm, block=tile)
+    dq, D, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], sc, block_mask=bm, block=tile)
+    dk, dv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], sc, block_mask=bm, block=tile)
+    empty = {0: slice(16, 24), 1: slice(32, 40)}
+    for h, sl in empty.items():
+        assert np.all(o[h, sl] == 0.0) and np.all(np.isneginf(lse[h, sl]))
+        assert np.all(dq[h, sl] == 0.0) and np.all(D[h, sl] == 0.0)
+        keep = [i for i in range(N) if not (sl.start <= i < sl.stop)]
+        q = _f64(x["q"][0, h, keep]).requires_grad_(True)
+        k = _f64(x["k"][0, h]).requires_grad_(True)
+        v = _f64(x["v"][0, h]).requires_grad_(True)
+        o_ref = torch.softmax((q @ k.T) * sc, dim=-1) @ v
+        o_ref.backward(_f64(x["do"][0, h, keep]))
+        assert np.max(np.abs(o[h, keep] - o_ref.detach().numpy())) < 1e-12
+        assert np.max(np.abs(dk[h] - k.grad.numpy())) < 1e-11
+        assert np.max(np.abs(dv[h] - v.grad.numpy())) < 1e-11
+
+
+def test_block_mask_shape_is_checked():
+    x = make_inputs(1, 2, 40, 8, seed=36)
+    with pytest.raises(ValueError):
+        oracle.forward(x["q"], x["k"], x["v"], 0.3, block_mask=np.ones((1, 4, 4), np.uint8), block=8)
+    with pytest.raises(ValueError):
+        oracle.forward(x["q"], x["k"], x["v"], 0.3, block_mask=np.ones((3, 5, 5), np.uint8), block=8)
