@@ -194,6 +194,35 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    float dropout_p, uint64_t seed, void* stream);
 
 /*
+ * Block-sparse attention ("FlashAttention for Efficient Training" section
+ * 3.2, Block-Sparse Attention Support: only the non-zero blocks of the
+ * attention matrix are computed).  block_mask is a device array of bytes
+ * [mask_heads][nt][nt], nt = ceil(N / 128), row-major; mask_heads is 1 (one
+ * mask for every head) or H (head h uses slice h).  A nonzero byte at
+ * [h][a][c] lets queries 128a..128a+127 see keys 128c..128c+127; a zero hides
+ * that whole block (its scores count as -inf).  The causal mask, if set,
+ * applies on top.  A query row that sees no key at all gets o = 0 and
+ * lse = -inf (the pages do not define this case; it is the zero-weight limit),
+ * and contributes nothing to dq, dk, dv; a key no query sees gets dk = dv = 0.
+ * Work and memory traffic scale with the number of visible blocks.
+ *  - strides: as fa_fwd_strided (4 entries: q, k, v, o) and fa_bwd_strided
+ *    (8 entries); NULL means dense [B,H,N,d] tensors.
+ *  - N is at most 4096 * 128 = 524288 (FA_ERR_TOO_LARGE beyond); a null
+ *    block_mask or mask_heads other than 1 or H is FA_ERR_INVALID_ARG.
+ *  - The backward must get the mask the forward used; the mask is read, not
+ *    retained, and must stay unchanged while the calls run on the stream.
+ *  - Other arguments, outputs, workspace and errors are those of
+ *    fa_fwd_strided and fa_bwd_strided.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                       int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                       const uint8_t* block_mask, int mask_heads, void* stream);
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                       void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d,
+                       float scale, int causal, float dropout_p, uint64_t seed, const uint8_t* block_mask,
+                       int mask_heads, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Debug export of the dropout mask: for each listed head bh = b*H + h
  * (heads[nheads]) and query row (rows[nrows]), writes the keep bit of every
  * key j < N to out[(hi * nrows + ri) * N + j] (1 = kept).  heads, rows and

@@ -29,7 +29,8 @@ FA_ERR_TOO_LARGE = -7
 
 EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
-           "fa_bwd_finalize", "fa_bwd_noalloc", "fa_dropout_mask", "fa_strerror",
+           "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
+           "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -71,6 +72,9 @@ def load() -> ctypes.CDLL:
         lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, SZ,
                                        vp]
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
+        lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I, vp]
+        lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I,
+                                           vp, SZ, vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
         lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
@@ -81,8 +85,9 @@ def load() -> ctypes.CDLL:
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
-        for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd, lib.fa_bwd_prepare, lib.fa_bwd_recompute,
-                   lib.fa_bwd_finalize, lib.fa_bwd_noalloc, lib.fa_dropout_mask, lib.fa_get_device_error,
+        for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
+                   lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
+                   lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
         _lib = lib
@@ -130,13 +135,31 @@ def _strides(*ts):
     return arr
 
 
+def _check_block_mask(m, q):
+    """Block mask: uint8 CUDA tensor [1 or H, nt, nt], nt = ceil(N / 128), dense."""
+    B, H, N, d = q.shape
+    nt = (N + 127) // 128
+    if not m.is_cuda or m.device != q.device:
+        raise ValueError("block_mask must be a CUDA tensor on the inputs' device")
+    if m.dtype not in (torch.uint8, torch.bool):
+        raise ValueError("block_mask must be uint8 or bool")
+    if m.dim() != 3 or m.shape[0] not in (1, H) or tuple(m.shape[1:]) != (nt, nt):
+        raise ValueError(f"block_mask must be [1 or {H}, {nt}, {nt}], got {tuple(m.shape)}")
+    if not m.is_contiguous():
+        raise ValueError("block_mask must be contiguous")
+    return m.view(torch.uint8) if m.dtype == torch.bool else m
+
+
 def _call(rc: int, what: str):
     if rc != FA_OK:
         raise FaError(rc, what)
 
 
-def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=None, stream=None):
-    """O and lse of exact attention via ``fa_fwd``."""
+def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=None, stream=None,
+        block_mask=None):
+    """O and lse of exact attention via ``fa_fwd_strided``, or
+    ``fa_fwd_blocksparse`` when a ``block_mask`` ([1 or H, nt, nt] uint8 over
+    128 x 128 blocks) is given."""
     _check_inputs(q, k, v)
     B, H, N, d = q.shape
     if scale is None:
@@ -146,6 +169,13 @@ def fwd(q, k, v, causal=False, scale=None, dropout_p=0.0, seed=0, o=None, lse=No
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check_inputs(q, o)
+    if block_mask is not None:
+        m = _check_block_mask(block_mask, q)
+        rc = load().fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _strides(q, k, v, o), B, H,
+                                       N, d, float(scale), int(bool(causal)), float(dropout_p), int(seed), _ptr(m),
+                                       int(m.shape[0]), _stream(stream))
+        _call(rc, "fa_fwd_blocksparse")
+        return o, lse
     rc = load().fa_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _strides(q, k, v, o), B, H, N, d,
                                float(scale), int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
     _call(rc, "fa_fwd")
@@ -183,8 +213,9 @@ def bwd_workspace_size(B, H, N, d) -> int:
 
 
 def bwd(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, dq=None, dk=None,
-        dv=None, workspace=None, stream=None):
-    """dQ, dK, dV via ``fa_bwd`` (allocates the workspace with torch if not given)."""
+        dv=None, workspace=None, stream=None, block_mask=None):
+    """dQ, dK, dV via ``fa_bwd_strided`` (or ``fa_bwd_blocksparse`` with the
+    forward's ``block_mask``); allocates the workspace with torch if not given."""
     _check_inputs(q, k, v, o, dout)
     B, H, N, d = q.shape
     if scale is None:
@@ -196,6 +227,15 @@ def bwd(q, k, v, o, dout, lse, causal=False, scale=None, dropout_p=0.0, seed=0, 
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check_inputs(q, dq, dk, dv)
+    if block_mask is not None:
+        m = _check_block_mask(block_mask, q)
+        rc = load().fa_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), _strides(q, k, v, o, dout, dq, dk, dv), B, H, N, d,
+                                       float(scale), int(bool(causal)), float(dropout_p), int(seed), _ptr(m),
+                                       int(m.shape[0]), _ptr(workspace),
+                                       int(workspace.numel() * workspace.element_size()), _stream(stream))
+        _call(rc, "fa_bwd_blocksparse")
+        return dq, dk, dv
     rc = load().fa_bwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                _ptr(dv), _strides(q, k, v, o, dout, dq, dk, dv), B, H, N, d, float(scale),
                                int(bool(causal)), float(dropout_p), int(seed), _ptr(workspace),

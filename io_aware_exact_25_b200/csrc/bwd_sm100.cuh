@@ -23,13 +23,18 @@
 //     causal).  Per step it computes, in tensor memory with keys on the lanes,
 //     S^T = K_j Q_i^T and dP^T = V_j dO_i^T, forms P^T and dS^T in registers,
 //     accumulates dV += P^T dO_i and dK += dS^T Q_i in tensor memory, and
-//     computes the dQ_i partial dS K_j, which a warpgroup adds into the fp32
-//     accumulator with vector atomics (red.global.add.v4.f32);
+//     computes the dQ_i partial dS K_j, which a warpgroup stages in shared
+//     memory and adds into the fp32 accumulator with bulk reductions;
 //  3. dQ = scale * accumulator, rounded to bf16.
+// Block-sparse mode ("FlashAttention for Efficient Training" section 3.2,
+// Block-Sparse Attention Support): the CTA of key tile j loops only over
+// the query tiles whose mask entry for j is nonzero (a bit set in shared
+// memory built by the producer warp); a key tile no query tile sees writes
+// dK = dV = 0, and dQ rows nobody reaches keep the zeroed accumulator.
 // Warp roles of the fused kernel:
 //   warps 0-3   P/dS for query columns 0-63 of the step   (TMEM lanes = keys)
 //   warps 4-7   P/dS for query columns 64-127
-//   warps 8-11  dQ read-out and atomic accumulation        (TMEM lanes = queries)
+//   warps 8-11  dQ read-out and accumulation               (TMEM lanes = queries)
 //   warp  12    tcgen05 MMA issue (one thread)
 //   warp  13    TMA producer (+ dropout row keys)
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
@@ -69,6 +74,10 @@ struct BwdArgs {
   float* lse2;    // [BH, Npad] scratch: lse * log2(e), +inf on padded rows
   float* drow;    // [BH, Npad] scratch: D_i, 0 on padded rows
   int* err;
+  // block-sparse (SPARSE kernels only): bmask[hm][qt][kt] != 0 lets query
+  // tile qt see key tile kt; hm = 0 when bmask_heads == 1, else the head
+  const uint8_t* bmask;
+  int bmask_heads;
 };
 
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -198,8 +207,11 @@ struct BwdLayout {
   // row_empty[2], s, dp, p, ds, dv, dk, dq, dq_free, drain
   static constexpr int kNumBars = 1 + 12 + 9;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  // block-sparse: the query-tile bit set and its count after the barriers
+  static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
+  static constexpr uint32_t kSmemSparse = kOffBits + kSparseWords * 4u + 16u;
   static_assert(kOffDQ % 1024 == 0, "staging tiles must be swizzle-aligned");
-  static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kSmemSparse <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
@@ -211,7 +223,7 @@ __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk
 // exponential on the FMA pipe (polynomial), the rest on MUFU.
 constexpr int kBwdPolyPairsOf8 = 0;
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -253,8 +265,11 @@ __global__ void __launch_bounds__(448, 1)
   const int bh = blockIdx.x - jt * BH;
   const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
   const int i_begin = CAUSAL ? jt : 0;
-  const int n_steps = nT - i_begin;
+  int n_steps = nT - i_begin;  // query tiles this CTA visits
   const int npad = nT * 128;
+  uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // SPARSE: query tiles that see jt
+  int* sparse_cnt = reinterpret_cast<int*>(qbits + kSparseWords);
+  const int nwords = (nT + 31) >> 5;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -284,17 +299,25 @@ __global__ void __launch_bounds__(448, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (SPARSE && warp == 13) {
+    // column jt of the mask: entry (i, jt) for i in [i_begin, nT)
+    const int hm = a.bmask_heads == 1 ? 0 : hh;
+    const uint8_t* col = a.bmask + (size_t)hm * nT * nT + jt;
+    const int3 c = build_bit_sets(col, nT, nullptr, 0, i_begin, nT, nwords, qbits, nullptr, lane);
+    if (lane == 0) sparse_cnt[0] = c.x;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, a.err};
   const bool run = *abort_flag == 0;
+  if (SPARSE) n_steps = sparse_cnt[0];
 
   if (run && warp == 13) {
     // ------------------------------------------------------ TMA producer
     const uint64_t pol_keep = policy_evict_last();
-    if (lane == 0) {
+    if (lane == 0 && n_steps > 0) {  // (a key tile no query tile sees loads nothing)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -309,8 +332,9 @@ __global__ void __launch_bounds__(448, 1)
     // waits are made warp-uniform with __all_sync, lane 0 issues the copies.
     int q_issued = 0, do_issued = 0;
     bool ok = true;
+    BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < n_steps && ok; ++it) {
-      const int i = i_begin + it;
+      const int i = SPARSE ? walk.next() : i_begin + it;
       // Q_i and dO_i: re-read by every key tile of the head -> keep in L2
       const int qs = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar_q_empty[qs], ((it >> 1) & 1) ^ 1u, ab))) break;
@@ -350,7 +374,7 @@ __global__ void __launch_bounds__(448, 1)
       }
       __syncwarp();
     }
-    if (lane == 0) {
+    if (lane == 0 && n_steps > 0) {
       // Every load issued must land before the CTA may exit.
       mbar_wait_drain(bar_kv, 0);
       for (int n = q_issued > 2 ? q_issued - 2 : 0; n < q_issued; ++n) mbar_wait_drain(&bar_q_full[n & 1], (n >> 1) & 1);
@@ -364,7 +388,7 @@ __global__ void __launch_bounds__(448, 1)
       constexpr uint32_t kIdTM = idesc_bf16(128, D, false, true);     // dV, dK: A in TMEM, B MN-major
       constexpr uint32_t kIdMM = idesc_bf16(128, D, true, true);      // dQ: both MN-major
       const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sDS = sbase + L::kOffDS;
-      bool ok = mbar_wait(bar_kv, 0, ab) && mbar_wait(&bar_q_full[0], 0, ab);
+      bool ok = n_steps > 0 && mbar_wait(bar_kv, 0, ab) && mbar_wait(&bar_q_full[0], 0, ab);
       bool issued_any = false;
       if (ok) {
         tc_fence_after();
@@ -475,7 +499,9 @@ __global__ void __launch_bounds__(448, 1)
         bulk_commit();
       }
     };
+    BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < n_steps; ++it) {
+      const int i = SPARSE ? walk.next() : i_begin + it;
       // the staging tiles are free once the previous step's reductions read them
       if (leader) {
         bulk_wait_read<0>();
@@ -484,7 +510,7 @@ __global__ void __launch_bounds__(448, 1)
       named_bar_sync(1, 128);
       if (*dq_flag == 0) break;
       tc_fence_after();
-      float* acc_tile = a.dq_acc + ((size_t)bh * nT + (i_begin + it)) * (size_t)(128 * D);
+      float* acc_tile = a.dq_acc + ((size_t)bh * nT + i) * (size_t)(128 * D);
       if (D == 64) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tQ, v0);
@@ -547,8 +573,9 @@ __global__ void __launch_bounds__(448, 1)
     const float sl2 = a.scale_log2;
     const bool key_ok = key < a.N;
     bool ok = true;
+    BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < n_steps; ++it) {
-      const int i = i_begin + it;
+      const int i = SPARSE ? walk.next() : i_begin + it;
       const uint32_t ph = it & 1;
       const int rs = it % L::kRowStages;
       const uint32_t rowbuf = sbase + L::kOffRow + rs * L::kRowStage;
@@ -694,7 +721,15 @@ __global__ void __launch_bounds__(448, 1)
       mbar_arrive(&bar_row_empty[rs]);
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK = scale * acc
-    if (ok && n_steps > 0 && mbar_wait(bar_dk, (n_steps - 1) & 1, ab)) {
+    if (SPARSE && n_steps == 0) {
+      // no query tile sees this key tile
+      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + (long long)key * a.dv_sn
+                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + (long long)key * a.dk_sn;
+      if (key_ok) {
+#pragma unroll
+        for (int c = 0; c < D; c += 8) st_global_v4(dst + c, 0u, 0u, 0u, 0u);
+      }
+    } else if (ok && n_steps > 0 && mbar_wait(bar_dk, (n_steps - 1) & 1, ab)) {
       tc_fence_after();
       const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
       const float mul = wg == 0 ? 1.f : a.scale;
@@ -725,15 +760,16 @@ __global__ void __launch_bounds__(448, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE>
 cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const BwdArgs& a, cudaStream_t st) {
   using L = BwdLayout<D, DROPOUT>;
-  auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
+  auto kern = bwd_kernel<D, CAUSAL, DROPOUT, SPARSE>;
+  const int smem = (int)(SPARSE ? L::kSmemSparse : L::kSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
-  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, mdo, a);
+  kern<<<(unsigned)grid, L::kThreads, smem, st>>>(mq, mk, mv, mdo, a);
   return cudaGetLastError();
 }
 
@@ -747,22 +783,25 @@ inline cudaError_t launch_bwd_prepare(const BwdArgs& a, int d, cudaStream_t st) 
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool SPARSE>
 cudaError_t launch_bwd_recompute_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                    const CUtensorMap& mdo, const BwdArgs& a, bool causal,
                                    bool dropout, cudaStream_t st) {
   if (causal)
-    return dropout ? launch_bwd_main<D, true, true>(mq, mk, mv, mdo, a, st)
-                   : launch_bwd_main<D, true, false>(mq, mk, mv, mdo, a, st);
-  return dropout ? launch_bwd_main<D, false, true>(mq, mk, mv, mdo, a, st)
-                 : launch_bwd_main<D, false, false>(mq, mk, mv, mdo, a, st);
+    return dropout ? launch_bwd_main<D, true, true, SPARSE>(mq, mk, mv, mdo, a, st)
+                   : launch_bwd_main<D, true, false, SPARSE>(mq, mk, mv, mdo, a, st);
+  return dropout ? launch_bwd_main<D, false, true, SPARSE>(mq, mk, mv, mdo, a, st)
+                 : launch_bwd_main<D, false, false, SPARSE>(mq, mk, mv, mdo, a, st);
 }
 
 inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                         const CUtensorMap& mdo, const BwdArgs& a, int d,
                                         bool causal, bool dropout, cudaStream_t st) {
-  return d == 64 ? launch_bwd_recompute_d<64>(mq, mk, mv, mdo, a, causal, dropout, st)
-                 : launch_bwd_recompute_d<128>(mq, mk, mv, mdo, a, causal, dropout, st);
+  if (a.bmask)
+    return d == 64 ? launch_bwd_recompute_d<64, true>(mq, mk, mv, mdo, a, causal, dropout, st)
+                   : launch_bwd_recompute_d<128, true>(mq, mk, mv, mdo, a, causal, dropout, st);
+  return d == 64 ? launch_bwd_recompute_d<64, false>(mq, mk, mv, mdo, a, causal, dropout, st)
+                 : launch_bwd_recompute_d<128, false>(mq, mk, mv, mdo, a, causal, dropout, st);
 }
 
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {

@@ -107,15 +107,17 @@ uint32_t keep_threshold(float p) {
   return (uint32_t)t;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT, bool SPLIT>
+template <int D, bool CAUSAL, bool DROPOUT, int MODE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                cudaStream_t st) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT, SPLIT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kSmem);
+  constexpr bool SPLIT = MODE == fa::kFwdSplit;
+  auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT, MODE>;
+  const int smem = (int)(MODE == fa::kFwdSparse ? L::kSmemSparse : L::kSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   const long long grid = (long long)a.B * a.H * ((a.N + 255) / 256) * (SPLIT ? a.num_splits : 1);
-  kern<<<(unsigned)grid, L::kThreads, L::kSmem, st>>>(mq, mk, mv, a);
+  kern<<<(unsigned)grid, L::kThreads, smem, st>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (SPLIT) {
@@ -126,14 +128,21 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return FA_OK;
 }
 
-template <int D, bool SPLIT>
+template <int D, int MODE>
 int dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                  bool causal, bool dropout, cudaStream_t st) {
   if (causal)
-    return dropout ? launch_fwd<D, true, true, SPLIT>(mq, mk, mv, a, st)
-                   : launch_fwd<D, true, false, SPLIT>(mq, mk, mv, a, st);
-  return dropout ? launch_fwd<D, false, true, SPLIT>(mq, mk, mv, a, st)
-                 : launch_fwd<D, false, false, SPLIT>(mq, mk, mv, a, st);
+    return dropout ? launch_fwd<D, true, true, MODE>(mq, mk, mv, a, st)
+                   : launch_fwd<D, true, false, MODE>(mq, mk, mv, a, st);
+  return dropout ? launch_fwd<D, false, true, MODE>(mq, mk, mv, a, st)
+                 : launch_fwd<D, false, false, MODE>(mq, mk, mv, a, st);
+}
+
+// Block-mask checks shared by the block-sparse entry points.
+int check_block_mask(const uint8_t* mask, int mask_heads, int H, int N) {
+  if (!mask || (mask_heads != 1 && mask_heads != H)) return FA_ERR_INVALID_ARG;
+  if ((N + 127) / 128 > fa::kMaxSparseTiles) return FA_ERR_TOO_LARGE;
+  return FA_OK;
 }
 
 size_t splitkv_bytes(int B, int H, int N, int d, int splits) {
@@ -194,10 +203,12 @@ namespace {
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides, int B,
              int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int num_splits,
-             void* workspace, size_t workspace_bytes, void* stream) {
+             void* workspace, size_t workspace_bytes, const uint8_t* bmask, int bmask_heads, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
+  if (bmask && (rc = check_block_mask(bmask, bmask_heads, H, N)) != FA_OK) return rc;
+  if (bmask && num_splits > 1) return FA_ERR_INVALID_ARG;
   if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
@@ -227,6 +238,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   a.num_splits = num_splits;
   a.part_o = nullptr;
   a.part_lse = nullptr;
+  a.bmask = bmask;
+  a.bmask_heads = bmask_heads;
   if (num_splits > 1) {
     a.part_o = static_cast<float*>(workspace);
     a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -236,11 +249,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
   const bool dropout = dropout_p > 0.f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bmask)
+    return d == 64 ? dispatch_fwd<64, fa::kFwdSparse>(mq, mk, mv, a, causal != 0, dropout, st)
+                   : dispatch_fwd<128, fa::kFwdSparse>(mq, mk, mv, a, causal != 0, dropout, st);
   if (num_splits > 1)
-    return d == 64 ? dispatch_fwd<64, true>(mq, mk, mv, a, causal != 0, dropout, st)
-                   : dispatch_fwd<128, true>(mq, mk, mv, a, causal != 0, dropout, st);
-  return d == 64 ? dispatch_fwd<64, false>(mq, mk, mv, a, causal != 0, dropout, st)
-                 : dispatch_fwd<128, false>(mq, mk, mv, a, causal != 0, dropout, st);
+    return d == 64 ? dispatch_fwd<64, fa::kFwdSplit>(mq, mk, mv, a, causal != 0, dropout, st)
+                   : dispatch_fwd<128, fa::kFwdSplit>(mq, mk, mv, a, causal != 0, dropout, st);
+  return d == 64 ? dispatch_fwd<64, fa::kFwdPlain>(mq, mk, mv, a, causal != 0, dropout, st)
+                 : dispatch_fwd<128, fa::kFwdPlain>(mq, mk, mv, a, causal != 0, dropout, st);
 }
 
 }  // namespace
@@ -248,7 +264,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
 int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
                    int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
                    void* stream) {
-  return fwd_impl(q, k, v, o, lse, strides, B, H, N, d, scale, causal, dropout_p, seed, 1, nullptr, 0, stream);
+  return fwd_impl(q, k, v, o, lse, strides, B, H, N, d, scale, causal, dropout_p, seed, 1, nullptr, 0, nullptr, 0,
+                  stream);
 }
 
 int fa_splitkv_suggest(int B, int H, int N, int d) {
@@ -277,7 +294,7 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   const fa_strides s = contiguous_strides(H, N, d);
   const fa_strides all[4] = {s, s, s, s};
   return fwd_impl(q, k, v, o, lse, all, B, H, N, d, scale, causal, dropout_p, seed, num_splits, workspace,
-                  workspace_bytes, stream);
+                  workspace_bytes, nullptr, 0, stream);
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -360,10 +377,12 @@ int bwd_prepare_impl(const void* o, const void* dout, const float* lse, const fa
 
 int bwd_recompute_impl(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
                        const fa_strides* s, int B, int H, int N, int d, float scale, int causal, float dropout_p,
-                       uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+                       uint64_t seed, void* workspace, size_t workspace_bytes, const uint8_t* bmask,
+                       int bmask_heads, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
+  if (bmask && (rc = check_block_mask(bmask, bmask_heads, H, N)) != FA_OK) return rc;
   if (!q || !k || !v || !dout || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dk, 16) ||
       !aligned(dv, 16))
@@ -381,6 +400,8 @@ int bwd_recompute_impl(const void* q, const void* k, const void* v, const void* 
   a.dv_sb = s[7].b;
   a.dv_sh = s[7].h;
   a.dv_sn = s[7].n;
+  a.bmask = bmask;
+  a.bmask_heads = bmask_heads;
   CUtensorMap mq, mk, mv, mdo;
   if ((rc = make_tile_map(&mq, q, B, H, N, d, s[0])) != FA_OK) return rc;
   if ((rc = make_tile_map(&mk, k, B, H, N, d, s[1])) != FA_OK) return rc;
@@ -428,7 +449,7 @@ int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* do
   fa_strides s[8];
   contiguous8(H, N, d, s);
   return bwd_recompute_impl(q, k, v, dout, dk, dv, s, B, H, N, d, scale, causal, dropout_p, seed, workspace,
-                            workspace_bytes, stream);
+                            workspace_bytes, nullptr, 0, stream);
 }
 
 int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
@@ -438,13 +459,16 @@ int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* wor
   return bwd_finalize_impl(dq, s, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
-int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                   void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d, float scale,
-                   int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
-                   void* stream) {
+namespace {
+
+int bwd_all_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d, float scale,
+                 int causal, float dropout_p, uint64_t seed, const uint8_t* bmask, int bmask_heads, void* workspace,
+                 size_t workspace_bytes, void* stream) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
+  if (bmask && (rc = check_block_mask(bmask, bmask_heads, H, N)) != FA_OK) return rc;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !strides) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
@@ -455,9 +479,46 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
   if ((rc = bwd_prepare_impl(o, dout, lse, strides, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK)
     return rc;
   if ((rc = bwd_recompute_impl(q, k, v, dout, dk, dv, strides, B, H, N, d, scale, causal, dropout_p, seed, workspace,
-                               workspace_bytes, stream)) != FA_OK)
+                               workspace_bytes, bmask, bmask_heads, stream)) != FA_OK)
     return rc;
   return bwd_finalize_impl(dq, strides, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+}  // namespace
+
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d, float scale,
+                   int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  return bwd_all_impl(q, k, v, o, dout, lse, dq, dk, dv, strides, B, H, N, d, scale, causal, dropout_p, seed, nullptr,
+                      0, workspace, workspace_bytes, stream);
+}
+
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                       int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                       const uint8_t* block_mask, int mask_heads, void* stream) {
+  fa_strides c[4];
+  if (!strides) {
+    for (int t = 0; t < 4; ++t) c[t] = contiguous_strides(H, N, d);
+    strides = c;
+  }
+  if (!block_mask && B > 0 && H > 0 && N > 0) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, strides, B, H, N, d, scale, causal, dropout_p, seed, 1, nullptr, 0, block_mask,
+                  mask_heads, stream);
+}
+
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                       void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d,
+                       float scale, int causal, float dropout_p, uint64_t seed, const uint8_t* block_mask,
+                       int mask_heads, void* workspace, size_t workspace_bytes, void* stream) {
+  fa_strides c[8];
+  if (!strides) {
+    contiguous8(H, N, d, c);
+    strides = c;
+  }
+  if (!block_mask && B > 0 && H > 0 && N > 0) return FA_ERR_INVALID_ARG;
+  return bwd_all_impl(q, k, v, o, dout, lse, dq, dk, dv, strides, B, H, N, d, scale, causal, dropout_p, seed,
+                      block_mask, mask_heads, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,

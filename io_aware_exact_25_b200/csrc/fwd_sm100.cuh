@@ -23,6 +23,14 @@
 // warps, after S_t(j) has completed, which implies that every earlier MMA of
 // the issuing thread -- O_t += P_t V(j-1) included -- has completed too.
 //
+// Block-sparse mode ("FlashAttention for Efficient Training" section 3.2,
+// Block-Sparse Attention Support): a byte mask over 128 x 128 blocks says
+// which key tiles each query tile sees.  The producer warp turns the CTA's two
+// mask rows into bit sets in shared memory; the K/V ring then streams only
+// the union of the two sets, each softmax warpgroup walks its own set, and
+// the MMA issuer skips the products of a tile its query tile does not see.
+// A query tile that sees no key tile writes O = 0 and lse = -inf.
+//
 // Online softmax in base 2: x = s * scale * log2(e); m is a running row
 // maximum that is only raised (and O, l rescaled) when the tile maximum
 // exceeds it by more than 8, i.e. a factor 256.  Every P and l use the same
@@ -50,11 +58,14 @@ struct FwdArgs {
   int num_splits;
   float* part_o;
   float* part_lse;
+  // block-sparse (SPARSE kernels only): bmask[hm][qt][kt] != 0 lets query
+  // tile qt see key tile kt; hm = 0 when bmask_heads == 1, else the head
+  const uint8_t* bmask;
+  int bmask_heads;
 };
 
-// Of every 8 pairs of probabilities, this many take the exponential on the
-// FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
-constexpr int kPolyPairsOf8 = 0;
+// Kernel variants: plain, split-KV, block-sparse.
+enum FwdMode : int { kFwdPlain = 0, kFwdSplit = 1, kFwdSparse = 2 };
 
 template <int D>
 struct FwdLayout {
@@ -67,14 +78,20 @@ struct FwdLayout {
   static constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
   static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  // block-sparse: two key-tile bit sets and three counts after the barriers
+  static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
+  static constexpr uint32_t kSmemSparse = kOffBits + 2u * kSparseWords * 4u + 16u;
   static constexpr uint32_t kColO = 256;  // O_t at kColO + D * t
+  static_assert(kSmemSparse <= 232448, "shared memory budget");
 };
 
-template <int D, bool CAUSAL, bool DROPOUT, bool SPLIT>
+template <int D, bool CAUSAL, bool DROPOUT, int MODE>
 __global__ void __launch_bounds__(320, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
   using L = FwdLayout<D>;
+  constexpr bool SPLIT = MODE == kFwdSplit;
+  constexpr bool SPARSE = MODE == kFwdSparse;
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -93,8 +110,6 @@ __global__ void __launch_bounds__(320, 1)
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   const uint32_t sbase = smem_u32(smem);
 
-  // Work tile.  For the causal mask the CTA with the most key tiles goes
-  // first (longest-processing-time order across the grid).
   // Work tile.  For the causal mask the CTA with the most key tiles goes
   // first (longest-processing-time order across the grid); heads are
   // interleaved, and the CTAs of a wave sweep the key tiles of their heads in
@@ -122,9 +137,14 @@ __global__ void __launch_bounds__(320, 1)
     j0 = split * chunk;
     span = max(0, min(end_max, j0 + chunk) - j0);
   }
-  const int nkv0 = max(0, min(end0, j0 + span) - j0);
-  const int nkv1 = max(0, min(end1, j0 + span) - j0);
-  const int nkv_max = nkv0 > nkv1 ? nkv0 : nkv1;
+  // steps of the K/V stream (nkv_max) and how many of them each Q tile uses
+  int nkv0 = max(0, min(end0, j0 + span) - j0);
+  int nkv1 = max(0, min(end1, j0 + span) - j0);
+  int nkv_max = nkv0 > nkv1 ? nkv0 : nkv1;
+  uint32_t* bits0 = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // SPARSE: key tiles of Q0
+  uint32_t* bits1 = bits0 + kSparseWords;                              // SPARSE: key tiles of Q1
+  int* sparse_cnt = reinterpret_cast<int*>(bits1 + kSparseWords);
+  const int nwords = (n_kv_all + 31) >> 5;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar_q[0], 1);
@@ -149,12 +169,27 @@ __global__ void __launch_bounds__(320, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (SPARSE && warp == 9) {
+    const int hm = a.bmask_heads == 1 ? 0 : hh;
+    const uint8_t* row0 = a.bmask + ((size_t)hm * n_kv_all + qt0) * n_kv_all;
+    const int3 c = build_bit_sets(row0, end0, act1 ? row0 + n_kv_all : nullptr, end1, 0, 1, nwords, bits0, bits1, lane);
+    if (lane == 0) {
+      sparse_cnt[0] = c.x;
+      sparse_cnt[1] = c.y;
+      sparse_cnt[2] = c.z;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, a.err};
   const bool run = *abort_flag == 0;
+  if (SPARSE) {
+    nkv0 = sparse_cnt[0];
+    nkv1 = sparse_cnt[1];
+    nkv_max = sparse_cnt[2];
+  }
 
   if (run && warp == 9) {
     // ------------------------------------------------------ TMA producer
@@ -164,7 +199,8 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tm_v);
       const uint64_t pol_keep = policy_evict_last();   // K/V: re-read by every Q tile of the head
       const uint64_t pol_once = policy_evict_first();  // Q: read once
-      for (int t = 0; t < 2; ++t) {
+      // (a CTA with no key tile to visit loads nothing)
+      for (int t = 0; t < 2 && nkv_max > 0; ++t) {
         if (t == 1 && !act1) break;
         mbar_arrive_expect_tx(&bar_q[t], L::kTile);
         for (int h = 0; h < D / 64; ++h)
@@ -175,7 +211,9 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
+      BitWalk walk(bits0, bits1, nwords);
       for (int j = 0; j < nkv_max && ok; ++j) {
+        const int kt = SPARSE ? walk.next() : j0 + j;  // key tile of this step
         for (int which = 0; which < 2; ++which) {
           if (!mbar_wait(&bar_kv_empty[stage], phase ^ 1u, ab)) {
             ok = false;
@@ -184,7 +222,7 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, (j0 + j) * 128, hh, bb,
+            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, kt * 128, hh, bb,
                         &bar_kv_full[stage], pol_keep);
           ++issued;
           if (++stage == L::kStages) {
@@ -194,8 +232,10 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // Every load issued must land before the CTA may exit.
-      mbar_wait_drain(&bar_q[0], 0);
-      if (act1) mbar_wait_drain(&bar_q[1], 0);
+      if (nkv_max > 0) {
+        mbar_wait_drain(&bar_q[0], 0);
+        if (act1) mbar_wait_drain(&bar_q[1], 0);
+      }
       const int first = issued > L::kStages ? issued - L::kStages : 0;
       for (int n = first; n < issued; ++n) mbar_wait_drain(&bar_kv_full[n % L::kStages], (n / L::kStages) & 1);
     }
@@ -208,11 +248,13 @@ __global__ void __launch_bounds__(320, 1)
     // needed between them.  The softmax publishes P_t in two halves (keys
     // 0-63, 64-127) so the product starts on the first half early.  K(j)
     // sits at ring position 2j, V(j) at 2j+1; stages are released in ring
-    // order.
+    // order.  A Q tile that does not see the key tile of a step (block-sparse)
+    // gets neither product for it; its P V product for its previous tile is
+    // still issued on the step after that tile.
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // S = Q K^T, both K-major
       constexpr uint32_t kIdO = idesc_bf16(128, D, false, true);     // O += P V, V is MN-major
-      bool ok = mbar_wait(&bar_q[0], 0, ab) && (!act1 || mbar_wait(&bar_q[1], 0, ab));
+      bool ok = nkv_max > 0 && mbar_wait(&bar_q[0], 0, ab) && (!act1 || mbar_wait(&bar_q[1], 0, ab));
       bool issued_any = false;
       auto stage_of = [](int pos) { return pos % L::kStages; };
       auto phase_of = [](int pos) { return (uint32_t)((pos / L::kStages) & 1); };
@@ -240,13 +282,25 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(&bar_pv[t]);
         return true;
       };
+      // does Q tile t see the key tile kt of step j?
+      auto sees = [&](int t, int j, int kt) -> bool {
+        if (SPARSE) return bit_set(t ? bits1 : bits0, kt);
+        return j < (t ? nkv1 : nkv0);
+      };
+      BitWalk walk(bits0, bits1, nwords);
+      int pv_count[2] = {0, 0};  // P V products issued per Q tile
+      bool prev[2] = {false, false};
       if (nkv_max == 0) {
-        ok = false;  // nothing to do in this split
+        ok = false;  // nothing to do in this split / block row
       } else if (ok && mbar_wait(&bar_kv_full[0], 0, ab)) {
         tc_fence_after();
         const uint32_t sK0 = sbase + L::kOffKV;
-        if (nkv0 > 0) issue_s(0, sK0);
-        if (nkv1 > 0) issue_s(1, sK0);
+        const int kt = SPARSE ? walk.next() : j0;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          prev[t] = sees(t, 0, kt);
+          if (prev[t]) issue_s(t, sK0);
+        }
         mma_commit(&bar_kv_empty[0]);
       } else {
         ok = false;
@@ -259,15 +313,16 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTile;
         const uint32_t sK = sbase + L::kOffKV + stage_of(posK) * L::kTile;
+        const int kt = SPARSE ? walk.next() : j0 + j;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const int nkv_t = t ? nkv1 : nkv0;
-          if (!ok || j - 1 >= nkv_t) continue;
-          if (!issue_pv(t, j - 1, sV)) {
+          if (!ok) continue;
+          if (prev[t] && !issue_pv(t, pv_count[t]++, sV)) {
             ok = false;
             continue;
           }
-          if (j < nkv_t) issue_s(t, sK);
+          prev[t] = sees(t, j, kt);
+          if (prev[t]) issue_s(t, sK);
         }
         if (!ok) break;
         mma_commit(&bar_kv_empty[stage_of(posV)]);  // V(j-1) consumed
@@ -281,7 +336,7 @@ __global__ void __launch_bounds__(320, 1)
           bool last_ok = true;
 #pragma unroll
           for (int t = 0; t < 2; ++t)
-            if (last_ok && j < (t ? nkv1 : nkv0)) last_ok = issue_pv(t, j, sV);
+            if (last_ok && prev[t]) last_ok = issue_pv(t, pv_count[t]++, sV);
           mma_commit(&bar_kv_empty[stage_of(posV)]);
         }
       }
@@ -307,7 +362,9 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t rkey = 0;
       if (DROPOUT) rkey = dropout_row_key(a.seed, (uint32_t)bb, (uint32_t)hh, (uint32_t)q_row);
       bool ok = true;
+      BitWalk walk(t ? bits1 : bits0, t ? bits1 : bits0, nwords);
       for (int j = 0; j < nkv; ++j) {
+        const int jg = SPARSE ? walk.next() : j0 + j;  // global key tile
         if (!mbar_wait(&bar_s[t], j & 1, ab)) {
           ok = false;
           break;
@@ -319,7 +376,6 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
-        const int jg = j0 + j;  // global key tile
         // key 128 jg + c is visible to query 128 (qt0 + t) + r iff c < lim;
         // only the diagonal tile (causal) or the ragged last tile masks
         int lim = 128;
@@ -425,7 +481,15 @@ __global__ void __launch_bounds__(320, 1)
       }
       // epilogue: O = O_t / l, lse = (m + log2 l) ln 2
       const bool in_range = q_row < a.N;
-      if (SPLIT && nkv == 0) {
+      if (SPARSE && nkv == 0) {
+        // the mask hides every key tile from this query tile
+        if (in_range && ok) {
+          __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)q_row * a.o_sn;
+#pragma unroll
+          for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+          a.lse[(size_t)bh * a.N + q_row] = -INFINITY;
+        }
+      } else if (SPLIT && nkv == 0) {
         // this split holds no key tile of this query tile: an empty partial
         if (in_range && ok) {
           float* prow = a.part_o + (((size_t)split * BH + bh) * a.N + q_row) * D;

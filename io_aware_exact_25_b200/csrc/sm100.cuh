@@ -464,4 +464,72 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
   return v;
 }
 
+// ---------------------------------------------------- block-sparse tile sets
+
+// Largest tile count block-sparse kernels handle (bit sets in shared
+// memory): N <= 4096 * 128.
+constexpr int kMaxSparseTiles = 4096;
+constexpr int kSparseWords = kMaxSparseTiles / 32;
+
+// Walks the set bits of (x | y) in ascending order; the caller never asks for
+// more indices than there are set bits.  Nothing is read before the first
+// next(), so kernels without bit sets may construct one.
+struct BitWalk {
+  const uint32_t* x;
+  const uint32_t* y;
+  int w, nwords;
+  uint32_t cur;
+  __device__ __forceinline__ BitWalk(const uint32_t* x_, const uint32_t* y_, int nwords_)
+      : x(x_), y(y_), w(-1), nwords(nwords_), cur(0u) {}
+  __device__ __forceinline__ int next() {
+    while (cur == 0u && w + 1 < nwords) {
+      ++w;
+      cur = x[w] | y[w];
+    }
+    const int b = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    return 32 * w + b;
+  }
+};
+
+__device__ __forceinline__ bool bit_set(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
+
+// One warp: bit sets of the nonzero bytes row[j * stride], begin <= j < end,
+// of up to two mask rows (row1 and bits1 may be null), written to bits0/bits1
+// (nwords words each).  Returns the popcounts of the two sets and of their
+// union.
+__device__ __forceinline__ int3 build_bit_sets(const uint8_t* row0, int end0, const uint8_t* row1, int end1,
+                                               int begin, long long stride, int nwords, uint32_t* bits0,
+                                               uint32_t* bits1, int lane) {
+  int c0 = 0, c1 = 0, cu = 0;
+  for (int w0 = 0; w0 < nwords; w0 += 4) {
+    uint8_t v0[4], v1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = 32 * (w0 + k) + lane;
+      v0[k] = (j >= begin && j < end0) ? __ldg(row0 + (long long)j * stride) : (uint8_t)0;
+      v1[k] = (row1 && j >= begin && j < end1) ? __ldg(row1 + (long long)j * stride) : (uint8_t)0;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t m0 = __ballot_sync(0xffffffffu, v0[k] != 0);
+      const uint32_t m1 = __ballot_sync(0xffffffffu, v1[k] != 0);
+      if (w0 + k < nwords) {
+        if (lane == 0) {
+          bits0[w0 + k] = m0;
+          if (bits1) bits1[w0 + k] = m1;
+        }
+        c0 += __popc(m0);
+        c1 += __popc(m1);
+        cu += __popc(m0 | m1);
+      }
+    }
+  }
+  return make_int3(c0, c1, cu);
+}
+
+// Of every 8 pairs of probabilities, this many take the exponential on the
+// FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
+constexpr int kPolyPairsOf8 = 0;
+
 }  // namespace fa

@@ -91,6 +91,47 @@ def workload_inputs(w: Workload) -> dict:
     return make_inputs(w.B, w.H, w.N, w.d, w.seed, w.qkv_scale, w.offset_norm)
 
 
+def block_mask(kind: str, H: int, N: int, seed: int = 0, block: int = 128) -> torch.Tensor:
+    """Seeded synthetic block mask, uint8 ``[H, nt, nt]`` with ``nt = ceil(N / block)``.
+
+    Structures of block-sparse attention patterns (the pages' section 3.2 on
+    block-sparse attention names no specific pattern):
+      * ``"random:<density>"`` -- each block kept with that probability,
+        drawn per head;
+      * ``"local:<w>,global:<g>"`` -- a band of ``w`` block diagonals on each
+        side of the main one plus the first ``g`` block rows and columns (a
+        sliding window with global tokens), the same for every head;
+      * ``"ones"`` / ``"zeros"``.
+    """
+    nt = (N + block - 1) // block
+    if kind == "ones":
+        return torch.ones((H, nt, nt), dtype=torch.uint8)
+    if kind == "zeros":
+        return torch.zeros((H, nt, nt), dtype=torch.uint8)
+    if kind.startswith("random:"):
+        g = torch.Generator().manual_seed(int(seed))
+        return (torch.rand((H, nt, nt), generator=g) < float(kind.split(":")[1])).to(torch.uint8)
+    if kind.startswith("local:"):
+        parts = dict(p.split(":") for p in kind.split(","))
+        w, gl = int(parts["local"]), int(parts.get("global", 0))
+        i = torch.arange(nt)
+        m = ((i[:, None] - i[None, :]).abs() <= w) | (i[:, None] < gl) | (i[None, :] < gl)
+        return m.to(torch.uint8).unsqueeze(0).expand(H, nt, nt).contiguous()
+    raise ValueError(f"unknown block mask kind {kind!r}")
+
+
+def visible_block_fraction(mask: torch.Tensor, causal: bool) -> float:
+    """Work of a block mask relative to the dense non-causal problem, counting
+    a diagonal block as half under the causal mask (the convention that makes
+    dense causal attention half of dense)."""
+    m = mask.to(torch.float64)
+    nt = m.shape[-1]
+    if causal:
+        w = torch.tril(torch.ones(nt, nt, dtype=torch.float64), -1) + 0.5 * torch.eye(nt, dtype=torch.float64)
+        m = m * w
+    return float(m.sum() / (m.shape[0] * nt * nt))
+
+
 def sample_rows(N: int, count: int, seed: int) -> list:
     """Sorted sample of ``count`` distinct rows of ``range(N)`` that always
     contains 0 and N-1, drawn from a generator seeded with ``1000 + seed``."""

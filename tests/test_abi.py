@@ -111,6 +111,25 @@ def test_splitkv_workspace_and_arguments(lib):
     assert lib.fa_splitkv_suggest(1, 1, 16384, 128) == 2       # 64 CTAs -> one wave of 128
 
 
+def test_blocksparse_arguments(lib):
+    args = (1, 3, 300, 64, 0.125, 0, 0.0, 0)
+    # null mask, or a mask shared by neither one head nor all H heads
+    assert lib.fa_fwd_blocksparse(16, 16, 16, 16, 16, None, *args, None, 1, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_blocksparse(16, 16, 16, 16, 16, None, *args, 16, 2, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_blocksparse(16, 16, 16, 16, 16, 16, 16, 16, 16, None, *args, 16, 0, 16, 1 << 30, None) \
+        == binding.FA_ERR_INVALID_ARG
+    # more than 4096 key tiles
+    big = (1, 1, 4096 * 128 + 1, 64, 0.125, 0, 0.0, 0)
+    assert lib.fa_fwd_blocksparse(16, 16, 16, 16, 16, None, *big, 16, 1, None) == binding.FA_ERR_TOO_LARGE
+    assert lib.fa_bwd_blocksparse(16, 16, 16, 16, 16, 16, 16, 16, 16, None, *big, 16, 1, 16, 1 << 40, None) \
+        == binding.FA_ERR_TOO_LARGE
+    # workspace still checked; empty problems are no-ops
+    assert lib.fa_bwd_blocksparse(16, 16, 16, 16, 16, 16, 16, 16, 16, None, *args, 16, 3, None, 0, None) \
+        == binding.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_blocksparse(None, None, None, None, None, None, 1, 1, 0, 64, 0.1, 0, 0.0, 0, None, 1,
+                                  None) == binding.FA_OK
+
+
 def test_empty_problems_are_noops(lib):
     # nothing to do: success without touching the (absent) device or pointers
     assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == binding.FA_OK

@@ -24,11 +24,18 @@ REL_L2 = 5e-3
 LSE_ABS = 1e-3
 
 
+def bf16_ulp(x):
+    """One bf16 ulp at |x|: 2^(e - 7) for |x| in [2^e, 2^(e+1))."""
+    _, e = np.frexp(np.abs(x))
+    return np.ldexp(1.0, e - 8)
+
+
 def _check(name, got, ref, exclude_rows=None):
     """Max |err| <= 2e-2 and relative L2 <= 5e-3.
 
-    Where |ref| >= 8 one bf16 ulp of the output (>= 2^-5 there) exceeds the
-    absolute bound, so the bound there is one ulp (2^-8 |ref|).  Rows listed
+    Where |ref| >= 4 one bf16 ulp of the output (2^-5 in [4, 8), doubling per
+    binade) exceeds the absolute bound, and rounding the exact value to bf16
+    alone may use half of it; the bound there is one bf16 ulp of |ref|.  Rows listed
     in ``exclude_rows`` (index into axis -2) are left out of the relative
     metric only: they are rows whose exact value is identically zero, where a
     relative error is undefined; they still meet the absolute bound.  For the
@@ -37,9 +44,11 @@ def _check(name, got, ref, exclude_rows=None):
     g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
     assert np.all(np.isfinite(g)), f"{name}: non-finite output"
     err = np.abs(g - ref)
-    bound = np.maximum(MAX_ABS, np.abs(ref) * 2.0 ** -8)
+    bound = np.maximum(MAX_ABS, bf16_ulp(ref))
     worst = np.unravel_index(np.argmax(err / bound), err.shape)
-    assert np.all(err <= bound), f"{name}: abs err {err[worst]:.3e} at {worst} (|ref| {abs(ref[worst]):.3e})"
+    assert np.all(err <= bound), (f"{name}: abs err {err[worst]:.3e} at {worst} (|ref| {abs(ref[worst]):.3e}), "
+                                  f"{int((err > bound).sum())} over, rel L2 "
+                                  f"{np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-300):.3e}")
     if exclude_rows:
         keep = np.ones(ref.shape[-2], bool)
         keep[list(exclude_rows)] = False
