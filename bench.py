@@ -146,18 +146,27 @@ def recorded_traffic(kernel: str, workload: str):
 
 # ------------------------------------------------------- oracle (CPU)
 
-def oracle_step(x, w, n_rows: int):
+def oracle_step(x, w, n_rows: int, mask=None):
     """fp64 oracle forward + full backward on the causal prefix of length
     n_rows of head (b=0, h=0): an exact sub-problem of the workload (causal
-    rows < n_rows see only keys < n_rows).  Returns (seconds, FLOPs)."""
+    rows < n_rows see only keys < n_rows), with the top-left corner of the
+    block mask if there is one.  Returns (seconds, FLOPs)."""
     import oracle
+    from io_aware_exact_25_b200.inputs import visible_block_fraction
     q, k, v, do = (x[n][:1, :1, :n_rows].contiguous() for n in ("q", "k", "v", "do"))
+    bm = None
+    frac = 0.5 if w.causal else 1.0
+    if mask is not None:
+        nt = (n_rows + 127) // 128
+        sub = mask[:1, :nt, :nt].contiguous()
+        bm = sub.numpy()
+        frac = visible_block_fraction(sub, w.causal)
     t0 = time.perf_counter()
-    oracle.forward(q, k, v, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
-    oracle.backward_q(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
-    oracle.backward_kv(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    oracle.forward(q, k, v, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed, block_mask=bm)
+    oracle.backward_q(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed, block_mask=bm)
+    oracle.backward_kv(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed, block_mask=bm)
     dt = time.perf_counter() - t0
-    f = 4.0 * n_rows * n_rows * w.d / (2.0 if w.causal else 1.0)
+    f = 4.0 * n_rows * n_rows * w.d * frac
     return dt, 3.5 * f
 
 
@@ -191,12 +200,20 @@ def run_reference(args, w):
     return 0
 
 
-def workload_config(w):
-    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
-                        f"{'causal' if w.causal else 'non-causal'} dropout={w.p_drop} bf16",
-            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "dropout_p": w.p_drop,
-            "l2": "inputs larger than L2 (Q, K, V, dO: 4 x 64 MiB per step > 126 MB L2)",
-            "parallelism": "replicas: each GPU runs its own B*H heads, no collective"}
+def workload_config(w, mask_kind=None, frac=None):
+    tensor_mib = w.B * w.H * w.N * w.d * 2 / 2 ** 20
+    cfg = {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
+                       f"{'causal' if w.causal else 'non-causal'} dropout={w.p_drop} bf16",
+           "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "dropout_p": w.p_drop,
+           "l2": (f"inputs larger than L2 (Q, K, V, dO: 4 x {tensor_mib:.0f} MiB per step > 126 MB L2)"
+                  if 4 * tensor_mib > 126 else
+                  f"inputs ({4 * tensor_mib:.0f} MiB) fit in L2: no flush between steps"),
+           "parallelism": "replicas: each GPU runs its own B*H heads, no collective"}
+    if mask_kind:
+        cfg["block_mask"] = mask_kind
+        cfg["visible_block_fraction"] = frac
+        cfg["workload"] += f" block-sparse {mask_kind} ({100 * frac:.1f}% of dense non-causal work)"
+    return cfg
 
 
 # ------------------------------------------------------------ our arm
@@ -220,6 +237,12 @@ def run_ours(args, w):
     x = workload_inputs(w)
     B, H, N, d = w.B, w.H, w.N, w.d
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    mask_cpu, mask, frac = None, None, None
+    if args.block_mask:
+        from io_aware_exact_25_b200.inputs import block_mask, visible_block_fraction
+        mask_cpu = block_mask(args.block_mask, H, N, seed=w.seed)
+        mask = mask_cpu.to(dev)
+        frac = visible_block_fraction(mask_cpu, w.causal)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -239,7 +262,10 @@ def run_ours(args, w):
     split_ws = torch.empty(max(split_ws_bytes, 16), dtype=torch.uint8, device=dev)
 
     def fwd():
-        if splits > 1:
+        if mask is not None:
+            check(lib.fa_fwd_blocksparse(P(q), P(k), P(v), P(o), P(lse), None, B, H, N, d, w.scale, causal, w.p_drop,
+                                         w.seed, P(mask), H, s), "fa_fwd_blocksparse")
+        elif splits > 1:
             check(lib.fa_fwd_splitkv(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, w.scale, causal, w.p_drop, w.seed,
                                      splits, P(split_ws), split_ws_bytes, s), "fa_fwd_splitkv")
         else:
@@ -250,6 +276,11 @@ def run_ours(args, w):
         check(lib.fa_bwd_prepare(P(o), P(do), P(lse), B, H, N, d, P(work), wsb, s), "fa_bwd_prepare")
 
     def bwd_recompute():
+        if mask is not None:
+            check(lib.fa_bwd_recompute_blocksparse(P(q), P(k), P(v), P(do), P(dk), P(dv), B, H, N, d, w.scale, causal,
+                                                   w.p_drop, w.seed, P(mask), H, P(work), wsb, s),
+                  "fa_bwd_recompute_blocksparse")
+            return
         check(lib.fa_bwd_recompute(P(q), P(k), P(v), P(do), P(dk), P(dv), B, H, N, d, w.scale, causal,
                                    w.p_drop, w.seed, P(work), wsb, s), "fa_bwd_recompute")
 
@@ -299,8 +330,10 @@ def run_ours(args, w):
 
     if args.no_extras:
         if rank == 0:
+            ffp = w.fwd_flops() if frac is None else 4.0 * B * H * N * N * d * frac
             print(json.dumps({"profiling_run": True, "workload": w.name, "splitkv": splits,
-                              "fwd_tflops": w.fwd_flops() / (per_stage_ms[0] * 1e-3) / 1e12,
+                              "block_mask": args.block_mask,
+                              "fwd_tflops": ffp / (per_stage_ms[0] * 1e-3) / 1e12,
                               "ms_per_step": elapsed_ms / args.steps,
                               "stage_ms": dict(zip([n for n, _ in stages], per_stage_ms))}), flush=True)
         if ws > 1:
@@ -319,9 +352,10 @@ def run_ours(args, w):
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
         do.copy_(hdo, non_blocking=True)
-        binding.fwd(q, k, v, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed, o=o, lse=lse)
+        binding.fwd(q, k, v, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed, o=o, lse=lse,
+                    block_mask=mask)
         binding.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
-                    dq=dq, dk=dk, dv=dv, workspace=work)
+                    dq=dq, dk=dk, dv=dv, workspace=work, block_mask=mask)
         ho.copy_(o, non_blocking=True)
         hlse.copy_(lse, non_blocking=True)
         hdq.copy_(dq, non_blocking=True)
@@ -350,6 +384,11 @@ def run_ours(args, w):
 
     if rank == 0:
         ff, fb = w.fwd_flops(), w.bwd_flops()
+        if frac is not None:
+            # block-sparse: FLOPs of the visible blocks only (diagonal blocks
+            # count half under the causal mask)
+            ff = 4.0 * B * H * N * N * d * frac
+            fb = 2.5 * ff
         ms_step = elapsed_ms / args.steps
         value = ws * (ff + fb) / (ms_step * 1e-3) / 1e12
         fwd_ms = per_stage_ms[0]
@@ -367,19 +406,19 @@ def run_ours(args, w):
                     "unit": "TFLOP/s", "frac": achieved / sustained,
                     "peak_note": f"bf16_tflops_sustained of {peak_kind} (kernel timed inside a long step loop)",
                     "frac_of_burst": achieved / burst, "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,
-                    "traffic": recorded_traffic(names[dom], w.name),
+                    "traffic": recorded_traffic(names[dom], w.name) if mask is None else None,
                     "algorithmic_flops_per_launch": dom_flops}
         else:
             roof = {"bound": "hbm", "kernel": names[dom], "achieved": None, "peak": None, "unit": "GB/s",
                     "frac": None, "traffic": None}
         # oracle baseline on the host cores (bounded sample of the same workload)
         import oracle
-        cpu_dt, cpu_f = oracle_step(x, w, args.cpu_rows)
+        cpu_dt, cpu_f = oracle_step(x, w, args.cpu_rows, mask_cpu)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w),
+            "config": workload_config(w, args.block_mask, frac),
             "fwd_tflops": ws * ff / (fwd_ms * 1e-3) / 1e12,
             "fwd_bwd_tflops": value,
             "frac_of_peak": {
@@ -392,7 +431,8 @@ def run_ours(args, w):
             "roofline": roof,
             "cpu_baseline": {"value": cpu_f / cpu_dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
                              "kind": "oracle",
-                             "sample": f"fp64 fwd+bwd of the causal prefix N={args.cpu_rows} of head (0,0) "
+                             "sample": f"fp64 fwd+bwd of the causal prefix N={args.cpu_rows} of head (0,0)"
+                                       f"{' with its block mask corner' if mask is not None else ''} "
                                        f"({cpu_dt:.1f} s)"},
             "e2e": {"value": ws * (ff + fb) * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -419,6 +459,9 @@ def main():
                     help="causal prefix length of the oracle baseline sample")
     ap.add_argument("--splitkv", type=int, default=0,
                     help="forward with fa_fwd_splitkv: number of splits (-1: suggested, 0: plain kernel)")
+    ap.add_argument("--block-mask", default=None,
+                    help="block-sparse run with this synthetic block mask, e.g. 'local:4,global:2' or "
+                         "'random:0.25' (io_aware_exact_25_b200.inputs.block_mask)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end and CPU-baseline legs (profiling runs)")
     ap.add_argument("--ref-rows", type=int, default=1024,
@@ -426,6 +469,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.block_mask and args.splitkv:
+        ap.error("--block-mask and --splitkv are separate forward variants")
     from io_aware_exact_25_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
     if args.impl == "reference":

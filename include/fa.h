@@ -221,6 +221,14 @@ int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* 
                        void* dq, void* dk, void* dv, const fa_strides* strides, int B, int H, int N, int d,
                        float scale, int causal, float dropout_p, uint64_t seed, const uint8_t* block_mask,
                        int mask_heads, void* workspace, size_t workspace_bytes, void* stream);
+/* The recompute stage of fa_bwd_blocksparse on dense tensors, for the staged
+ * backward: fa_bwd_prepare, this, fa_bwd_finalize in order is exactly
+ * fa_bwd_blocksparse with strides == NULL.  Arguments as fa_bwd_recompute
+ * plus the block mask. */
+int fa_bwd_recompute_blocksparse(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                                 int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                                 const uint8_t* block_mask, int mask_heads, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /*
  * Debug export of the dropout mask: for each listed head bh = b*H + h

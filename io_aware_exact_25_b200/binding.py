@@ -30,6 +30,7 @@ FA_ERR_TOO_LARGE = -7
 EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
+           "fa_bwd_recompute_blocksparse",
            "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -75,6 +76,8 @@ def load() -> ctypes.CDLL:
         lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I, vp]
         lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I,
                                            vp, SZ, vp]
+        lib.fa_bwd_recompute_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, I, vp, SZ,
+                                                     vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
         lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
@@ -87,7 +90,8 @@ def load() -> ctypes.CDLL:
         lib.fa_get_device_error.argtypes = [vp]
         for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
                    lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
-                   lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_dropout_mask, lib.fa_get_device_error,
+                   lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
+                   lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
         _lib = lib

@@ -452,6 +452,17 @@ int fa_bwd_recompute(const void* q, const void* k, const void* v, const void* do
                             workspace_bytes, nullptr, 0, stream);
 }
 
+int fa_bwd_recompute_blocksparse(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                                 int B, int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed,
+                                 const uint8_t* block_mask, int mask_heads, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  fa_strides s[8];
+  contiguous8(H, N, d, s);
+  if (!block_mask && B > 0 && H > 0 && N > 0) return FA_ERR_INVALID_ARG;
+  return bwd_recompute_impl(q, k, v, dout, dk, dv, s, B, H, N, d, scale, causal, dropout_p, seed, workspace,
+                            workspace_bytes, block_mask, mask_heads, stream);
+}
+
 int fa_bwd_finalize(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
                     void* stream) {
   fa_strides s[8];

@@ -184,3 +184,29 @@ def test_autograd_wrapper_with_block_mask(cuda_device):
     rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], sc, causal=True, block_mask=bm)
     _check("O", o.transpose(1, 2), ro)
     _check("dQ", q.grad.transpose(1, 2), rdq)
+
+
+def test_staged_blocksparse_backward_equals_one_call(cuda_device):
+    """fa_bwd_prepare + fa_bwd_recompute_blocksparse + fa_bwd_finalize is
+    fa_bwd_blocksparse."""
+    B, H, N, d = 1, 2, 700, 128
+    x = make_inputs(B, H, N, d, seed=86)
+    xd = {n: t.to(cuda_device) for n, t in x.items()}
+    mask = block_mask("random:0.6", H, N, seed=87).to(cuda_device)
+    sc = 1.0 / math.sqrt(d)
+    o, lse = binding.fwd(xd["q"], xd["k"], xd["v"], causal=True, scale=sc, block_mask=mask)
+    dq1, dk1, dv1 = binding.bwd(xd["q"], xd["k"], xd["v"], o, xd["do"], lse, causal=True, scale=sc,
+                                block_mask=mask)
+    lib = binding.load()
+    wsb = binding.bwd_workspace_size(B, H, N, d)
+    work = torch.empty(wsb, dtype=torch.uint8, device=cuda_device)
+    dq2, dk2, dv2 = (torch.empty_like(xd["q"]) for _ in range(3))
+    s = torch.cuda.current_stream().cuda_stream
+    P = binding._ptr
+    assert lib.fa_bwd_prepare(P(o), P(xd["do"]), P(lse), B, H, N, d, P(work), wsb, s) == 0
+    assert lib.fa_bwd_recompute_blocksparse(P(xd["q"]), P(xd["k"]), P(xd["v"]), P(xd["do"]), P(dk2), P(dv2), B, H, N,
+                                            d, sc, 1, 0.0, 0, P(mask), H, P(work), wsb, s) == 0
+    assert lib.fa_bwd_finalize(P(dq2), B, H, N, d, sc, P(work), wsb, s) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    assert (dq1.float() - dq2.float()).abs().max().item() <= 2e-2
