@@ -40,9 +40,9 @@
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
 // [0,32) and [64,96); R_dP [128,256) dP^T fp32, then dS^T bf16 in [128,160)
 // and [192,224), then the dQ partial (fp32, D columns); dV at 256, dK at
-// 256 + D.  MMA order per step: dP(i), dV(i), dK(i), dQ(i), S(i+1); dP(i)
-// runs while the softmax warps form P(i), and the dQ read-out of one step
-// overlaps the next step's S and P.
+// 256 + D.  MMA order per step: dP(i), dV(i), S(i+1), dK(i), dQ(i); dP(i)
+// runs while the softmax warps form P(i), S(i+1) while they form dS(i), and
+// the dQ read-out of one step overlaps the next step's P.
 #pragma once
 
 #include "dropout_hash.cuh"
@@ -400,12 +400,14 @@ __global__ void __launch_bounds__(448, 1)
         mma_commit(bar_s);
         issued_any = true;
       }
-      // Per step: dP(i), dV(i), dK(i), dQ(i), S(i+1).  dP(i) overwrites the
+      // Per step: dP(i), dV(i), S(i+1), dK(i), dQ(i).  dP(i) overwrites the
       // dQ(i-1) partial and waits for the dQ warpgroup to have read it; it then
-      // runs while the softmax warps form P(i).  dQ(i) overwrites the columns
-      // holding dS^T(i), which dK(i) reads, and S(i+1) those holding P^T(i),
-      // which dV(i) reads; each is queued behind its reader and the tensor core
-      // executes one thread's MMAs in order, so neither needs a wait.
+      // runs while the softmax warps form P(i).  S(i+1) overwrites the columns
+      // holding P^T(i), which dV(i) reads, and dQ(i) those holding dS^T(i),
+      // which dK(i) reads; each is queued behind its reader and the tensor core
+      // executes one thread's MMAs in order, so neither needs a wait.  S(i+1)
+      // goes right behind dV(i) so it runs while the softmax warps form dS(i),
+      // and P(i+1) can start as soon as dS(i) is done.
       for (int it = 0; it < n_steps && ok; ++it) {
         const uint32_t ph = it & 1;
         const int qs = it & 1;
@@ -429,6 +431,18 @@ __global__ void __launch_bounds__(448, 1)
           mma_ts(tmem + L::kColDV, tmem + L::kColS + packed_col(kk), desc_mnmajor(sDO, kk, L::kHalf), kIdTM,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar_do_empty[ds_]);
+        // S^T for the next step (behind dV, which reads P^T from R_S)
+        if (it + 1 < n_steps) {
+          const int qn = (it + 1) & 1;
+          if (!mbar_wait(&bar_q_full[qn], ((it + 1) >> 1) & 1, ab)) break;
+          tc_fence_after();
+          const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQn, kk, L::kHalf), kIdKK,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_s);
+        }
         // dK += dS^T Q_i
         if (!mbar_wait(bar_ds, ph, ab)) break;
         tc_fence_after();
@@ -444,18 +458,6 @@ __global__ void __launch_bounds__(448, 1)
                  kk > 0 ? 1u : 0u);
         mma_commit(bar_dq);
         mma_commit(&bar_q_empty[qs]);
-        // S^T for the next step (behind dV, which read P^T from R_S)
-        if (it + 1 < n_steps) {
-          const int qn = (it + 1) & 1;
-          if (!mbar_wait(&bar_q_full[qn], ((it + 1) >> 1) & 1, ab)) break;
-          tc_fence_after();
-          const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQn, kk, L::kHalf), kIdKK,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(bar_s);
-        }
       }
       if (issued_any) {
         mma_commit(bar_drain);
