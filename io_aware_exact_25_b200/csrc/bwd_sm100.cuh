@@ -104,42 +104,53 @@ inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, 
 
 // ------------------------------------------------------------ row pass
 
-// One warp per (padded) row: D_i = sum_c dO_ic O_ic in fp32 and lse2_i; then
-// the whole dQ accumulator is set to zero.
+// D_i = sum_c dO_ic O_ic in fp32 and lse2_i for every (padded) row, then the
+// whole dQ accumulator is set to zero.  HBM-bound: a row is read by D / 8
+// lanes with 16-byte loads, and each warp keeps four groups of rows in flight.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, int npad) {
-  constexpr int kPer = D / 32;  // elements per lane
+  constexpr int kTpr = D * 2 / 16;  // lanes per row
+  constexpr int kRpw = 32 / kTpr;   // rows per warp per group
+  constexpr int kU = 4;             // groups in flight
   const long long rows = (long long)BH * npad;
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kTpr, part = lane - sub * kTpr;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long r = warp0; r < rows; r += nwarps) {
-    const int bh = (int)(r / npad);
-    const int i = (int)(r - (long long)bh * npad);
-    if (i < a.N) {
-      const int b_ = bh / a.H, h_ = bh - b_ * a.H;
-      const __nv_bfloat16* orow = a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + lane * kPer;
-      const __nv_bfloat16* drow = a.dout + b_ * a.do_sb + h_ * a.do_sh + (long long)i * a.do_sn + lane * kPer;
-      float acc = 0.f;
-      if (kPer == 4) {
-        const uint2 ov = *reinterpret_cast<const uint2*>(orow);
-        const uint2 dv = *reinterpret_cast<const uint2*>(drow);
-        acc = bf16_lo(ov.x) * bf16_lo(dv.x) + bf16_hi(ov.x) * bf16_hi(dv.x) + bf16_lo(ov.y) * bf16_lo(dv.y) +
-              bf16_hi(ov.y) * bf16_hi(dv.y);
-      } else {
-        const uint32_t ov = *reinterpret_cast<const uint32_t*>(orow);
-        const uint32_t dv = *reinterpret_cast<const uint32_t*>(drow);
-        acc = bf16_lo(ov) * bf16_lo(dv) + bf16_hi(ov) * bf16_hi(dv);
-      }
+  for (long long r0 = warp0 * (kRpw * kU); r0 < rows; r0 += nwarps * (kRpw * kU)) {
+    uint4 ov[kU], dv[kU];
 #pragma unroll
-      for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-      if (lane == 0) {
-        a.drow[r] = acc;
-        a.lse2[r] = a.lse[(size_t)bh * a.N + i] * 1.4426950408889634f;
+    for (int u = 0; u < kU; ++u) {
+      ov[u] = make_uint4(0u, 0u, 0u, 0u);
+      dv[u] = make_uint4(0u, 0u, 0u, 0u);
+      const long long r = r0 + u * kRpw + sub;
+      if (r < rows) {
+        const int bh = (int)(r / npad);
+        const int i = (int)(r - (long long)bh * npad);
+        if (i < a.N) {
+          const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+          ov[u] = *reinterpret_cast<const uint4*>(a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + 8 * part);
+          dv[u] = *reinterpret_cast<const uint4*>(a.dout + b_ * a.do_sb + h_ * a.do_sh + (long long)i * a.do_sn +
+                                                  8 * part);
+        }
       }
-    } else if (lane == 0) {
-      a.drow[r] = 0.f;
-      a.lse2[r] = INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const uint32_t o4[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+      const uint32_t d4[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc += bf16_lo(o4[e]) * bf16_lo(d4[e]) + bf16_hi(o4[e]) * bf16_hi(d4[e]);
+#pragma unroll
+      for (int s = kTpr / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+      const long long r = r0 + u * kRpw + sub;
+      if (part == 0 && r < rows) {
+        const int bh = (int)(r / npad);
+        const int i = (int)(r - (long long)bh * npad);
+        a.drow[r] = i < a.N ? acc : 0.f;
+        a.lse2[r] = i < a.N ? a.lse[(size_t)bh * a.N + i] * 1.4426950408889634f : INFINITY;
+      }
     }
   }
   const long long n4 = (long long)BH * npad * D / 4;

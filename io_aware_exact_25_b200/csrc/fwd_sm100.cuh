@@ -67,6 +67,10 @@ struct FwdArgs {
 // Kernel variants: plain, split-KV, block-sparse.
 enum FwdMode : int { kFwdPlain = 0, kFwdSplit = 1, kFwdSparse = 2 };
 
+// Of every 8 pairs of probabilities, this many take the exponential on the
+// FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
+constexpr int kPolyPairsOf8 = 0;
+
 template <int D>
 struct FwdLayout {
   static constexpr int kThreads = 320;

@@ -502,8 +502,4 @@ __device__ __forceinline__ int3 build_bit_sets(const uint8_t* row0, int end0, co
   return make_int3(c0, c1, cu);
 }
 
-// Of every 8 pairs of probabilities, this many take the exponential on the
-// FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
-constexpr int kPolyPairsOf8 = 0;
-
 }  // namespace fa
