@@ -22,7 +22,8 @@
 //     head, looping over the 128-row query tiles i that see it (i >= j when
 //     causal).  Per step it computes, in tensor memory with keys on the lanes,
 //     S^T = K_j Q_i^T and dP^T = V_j dO_i^T, forms P^T and dS^T in registers,
-//     accumulates dV += P^T dO_i and dK += dS^T Q_i in tensor memory, and
+//     accumulates dV += P^T dO_i (P^T from tensor memory) and dK += dS^T Q_i
+//     (dS from shared memory) in tensor memory, and
 //     computes the dQ_i partial dS K_j, which a warpgroup stages in shared
 //     memory and adds into the fp32 accumulator with bulk reductions;
 //  3. dQ = scale * accumulator, rounded to bf16.
@@ -38,11 +39,11 @@
 //   warp  12    tcgen05 MMA issue (one thread)
 //   warp  13    TMA producer (+ dropout row keys)
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
-// [0,32) and [64,96); R_dP [128,256) dP^T fp32, then dS^T bf16 in [128,160)
-// and [192,224), then the dQ partial (fp32, D columns); dV at 256, dK at
-// 256 + D.  MMA order per step: dP(i), dV(i), S(i+1), dK(i), dQ(i); dP(i)
-// runs while the softmax warps form P(i), S(i+1) while they form dS(i), and
-// the dQ read-out of one step overlaps the next step's P.
+// [0,32) and [64,96); R_dP [128,256) dP^T fp32, then the dQ partial (fp32,
+// D columns); dV at 256, dK at 256 + D.  dS goes to shared memory only.  MMA
+// order per step: dP(i), dV(i), S(i+1), dQ(i), dK(i); dP(i) runs while the
+// softmax warps form P(i), S(i+1) while they form dS(i), and the dQ read-out
+// of one step overlaps dK and the next step's P.
 #pragma once
 
 #include "dropout_hash.cuh"
@@ -226,7 +227,7 @@ struct BwdLayout {
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
-// TMEM column of the packed bf16 operand slice kk (16 queries) written by the
+// TMEM column of the packed bf16 P^T slice kk (16 queries) written by the
 // two P/dS warpgroups: queries 0-63 at [0,32), 64-127 at [64,96).
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
 
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdKK = idesc_bf16(128, 128, false, false);  // S^T, dP^T: both operands K-major
-      constexpr uint32_t kIdTM = idesc_bf16(128, D, false, true);     // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t kIdTM = idesc_bf16(128, D, false, true);     // dV, dK: A K-major, B MN-major
       constexpr uint32_t kIdMM = idesc_bf16(128, D, true, true);      // dQ: both MN-major
       const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sDS = sbase + L::kOffDS;
       bool ok = n_steps > 0 && mbar_wait(bar_kv, 0, ab) && mbar_wait(&bar_q_full[0], 0, ab);
@@ -411,14 +412,16 @@ __global__ void __launch_bounds__(448, 1)
         mma_commit(bar_s);
         issued_any = true;
       }
-      // Per step: dP(i), dV(i), S(i+1), dK(i), dQ(i).  dP(i) overwrites the
+      // Per step: dP(i), dV(i), S(i+1), dQ(i), dK(i).  dP(i) overwrites the
       // dQ(i-1) partial and waits for the dQ warpgroup to have read it; it then
       // runs while the softmax warps form P(i).  S(i+1) overwrites the columns
-      // holding P^T(i), which dV(i) reads, and dQ(i) those holding dS^T(i),
-      // which dK(i) reads; each is queued behind its reader and the tensor core
-      // executes one thread's MMAs in order, so neither needs a wait.  S(i+1)
-      // goes right behind dV(i) so it runs while the softmax warps form dS(i),
-      // and P(i+1) can start as soon as dS(i) is done.
+      // holding P^T(i), which dV(i) reads; it is queued behind its reader and
+      // the tensor core executes one thread's MMAs in order, so it needs no
+      // wait.  S(i+1) goes right behind dV(i) so it runs while the softmax
+      // warps form dS(i), and P(i+1) can start as soon as dS(i) is done.  dQ(i)
+      // and dK(i) both read dS from shared memory (dS^T for dK is the same tile
+      // read K-major); dQ(i) goes first so its read-out, which gates dP(i+1),
+      // starts while dK(i) runs.
       for (int it = 0; it < n_steps && ok; ++it) {
         const uint32_t ph = it & 1;
         const int qs = it & 1;
@@ -454,20 +457,20 @@ __global__ void __launch_bounds__(448, 1)
                    kk > 0 ? 1u : 0u);
           mma_commit(bar_s);
         }
-        // dK += dS^T Q_i
+        // dQ_i partial = dS K_j into R_dP (the softmax warps have read dP^T(i))
         if (!mbar_wait(bar_ds, ph, ab)) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::kColDK, tmem + L::kColDP + packed_col(kk), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_dk);
-        // dQ_i partial = dS K_j into R_dP (behind dK, which read dS^T there)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
                  kk > 0 ? 1u : 0u);
         mma_commit(bar_dq);
+        // dK += dS^T Q_i, A = the shared dS tile read K-major (rows = keys)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::kColDK, desc_kmajor(sDS, kk, L::kHalf), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_dk);
         mma_commit(&bar_q_empty[qs]);
       }
       if (issued_any) {
@@ -581,7 +584,6 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t tS = tmem + lane_off + L::kColS + col0;
     const uint32_t tDP = tmem + lane_off + L::kColDP + col0;
     const uint32_t tPst = tmem + lane_off + L::kColS + 64u * wg;   // packed P^T (32 columns)
-    const uint32_t tDSst = tmem + lane_off + L::kColDP + 64u * wg; // packed dS^T
     const uint32_t sDSrow = sbase + L::kOffDS + wg * L::kHalf + jr * 128;
     const float sl2 = a.scale_log2;
     const bool key_ok = key < a.N;
@@ -682,8 +684,8 @@ __global__ void __launch_bounds__(448, 1)
         ok = false;
         break;
       }
-      // the previous dQ partial read sDS; wait for it before overwriting
-      if (it > 0 && !mbar_wait(bar_dq, ph ^ 1u, ab)) {
+      // dQ(i-1) and dK(i-1) read sDS; wait for the later one before overwriting
+      if (it > 0 && !mbar_wait(bar_dk, ph ^ 1u, ab)) {
         ok = false;
         break;
       }
@@ -717,9 +719,9 @@ __global__ void __launch_bounds__(448, 1)
             pk[2 * c2 + e2] = pack_bf16x2(ds0, ds1);
           }
         }
-        tmem_st16(tDSst + 16u * hf, pk);
-        // shared-memory copy (A operand of dQ = dS K): row jr of this half,
-        // 16-byte chunks XOR-swizzled by (jr mod 8)
+        // dS into shared memory (A operand of dQ = dS K and, read K-major, of
+        // dK = dS^T Q): row jr of this half, 16-byte chunks XOR-swizzled by
+        // (jr mod 8)
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const uint32_t chunk = (uint32_t)(4 * hf + q8);
@@ -728,7 +730,6 @@ __global__ void __launch_bounds__(448, 1)
         }
       }
       fence_proxy_async_smem();
-      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
       mbar_arrive(&bar_row_empty[rs]);
