@@ -340,41 +340,65 @@ def run_ours(args, w):
             dist.destroy_process_group()
         return 0
 
-    # end to end: pinned host inputs -> device, fwd + bwd, results -> pinned host
+    # end to end through the public API: every step copies its inputs from
+    # pinned host memory to the device, runs binding.fwd + binding.bwd and
+    # copies every result back.  Uploads, compute and downloads run on three
+    # streams over two sets of device buffers, so step k+1's upload and step
+    # k-1's download overlap step k's compute (the PCIe link is full duplex).
     hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
-    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
-    hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hlse))
+    nbuf = 2
+    d_in = [{"q": q, "k": k, "v": v, "do": do}] + [
+        {n: torch.empty_like(q) for n in ("q", "k", "v", "do")} for _ in range(nbuf - 1)]
+    d_out = [{"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}] + [
+        {"o": torch.empty_like(q), "lse": torch.empty_like(lse), "dq": torch.empty_like(q),
+         "dk": torch.empty_like(q), "dv": torch.empty_like(q)} for _ in range(nbuf - 1)]
+    h_out = [{n: torch.empty_like(t, device="cpu").pin_memory() for n, t in d_out[0].items()} for _ in range(nbuf)]
+    d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
+    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_cmp = stream
+    ev_up, ev_cmp, ev_dn = ([torch.cuda.Event() for _ in range(nbuf)] for _ in range(3))
+    for evs, st in ((ev_up, s_up), (ev_cmp, s_cmp), (ev_dn, s_dn)):
+        for e in evs:
+            e.record(st)
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        do.copy_(hdo, non_blocking=True)
-        binding.fwd(q, k, v, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed, o=o, lse=lse,
-                    block_mask=mask)
-        binding.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
-                    dq=dq, dk=dk, dv=dv, workspace=work, block_mask=mask)
-        ho.copy_(o, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
-        hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True)
-        hdv.copy_(dv, non_blocking=True)
+    def e2e_step(kstep):
+        bi = kstep % nbuf
+        din, dout, hout = d_in[bi], d_out[bi], h_out[bi]
+        s_up.wait_event(ev_cmp[bi])  # step k-2 finished reading these inputs
+        with torch.cuda.stream(s_up):
+            for n, h in (("q", hq), ("k", hk), ("v", hv), ("do", hdo)):
+                din[n].copy_(h, non_blocking=True)
+        ev_up[bi].record(s_up)
+        s_cmp.wait_event(ev_up[bi])
+        s_cmp.wait_event(ev_dn[bi])  # step k-2's results are on the host
+        binding.fwd(din["q"], din["k"], din["v"], causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
+                    o=dout["o"], lse=dout["lse"], block_mask=mask, stream=s_cmp)
+        binding.bwd(din["q"], din["k"], din["v"], dout["o"], din["do"], dout["lse"], causal=w.causal, scale=w.scale,
+                    dropout_p=w.p_drop, seed=w.seed, dq=dout["dq"], dk=dout["dk"], dv=dout["dv"], workspace=work,
+                    block_mask=mask, stream=s_cmp)
+        ev_cmp[bi].record(s_cmp)
+        s_dn.wait_event(ev_cmp[bi])
+        with torch.cuda.stream(s_dn):
+            for n, t in dout.items():
+                hout[n].copy_(t, non_blocking=True)
+        ev_dn[bi].record(s_dn)
 
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(3):
-        e2e_step()
+    for kstep in range(3):
+        e2e_step(kstep)
     barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_up)
+    for kstep in range(e2e_steps):
+        e2e_step(kstep)
+    e1.record(s_dn)  # the last download follows every upload and every compute
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error in the end-to-end run")
 
     # max over ranks
     from io_aware_exact_25_b200.replicas import max_over_ranks
@@ -436,7 +460,8 @@ def run_ours(args, w):
                                        f"({cpu_dt:.1f} s)"},
             "e2e": {"value": ws * (ff + fb) * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "binding.fwd/binding.bwd (C ABI) with pinned host buffers"},
+                    "api": "binding.fwd/binding.bwd (C ABI) with pinned host buffers; uploads, compute and "
+                           "downloads on three streams over two device buffer sets"},
             "gpu_launches": args.steps * (len(stages) + (1 if splits > 1 else 0)),
             "splitkv": splits,
             "clocks": clocks,
