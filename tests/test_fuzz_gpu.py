@@ -1,0 +1,139 @@
+"""Seeded random sweep of problem shapes and options against the fp64 oracle (GPU).
+
+Each case draws B, H, N, d, the scale, causal, dropout, the tensor layout
+(dense or the (batch, seq_len, num_heads, head_dim) view) and the variant
+(plain, block-sparse with a random block mask, or split-KV forward) from one
+seeded generator, runs the CUDA path through the C ABI and compares every
+element with the oracle.  At the workloads' operating point (scale at most
+1/sqrt(d), dropout at most 0.1) the bar is the parity bar of every other test:
+max |err| <= 2e-2 (one bf16 ulp of |ref| where that is larger) and relative
+L2 <= 5e-3 for O, dQ, dK, dV, lse within 1e-3.  Draws beyond it (scale up to
+1.5/sqrt(d), dropout 0.3) enlarge the bf16 rounding of dS and of the stored O
+that early causal rows concentrate on a few keys; there the absolute bound is
+doubled and the relative bound kept, which still fails any indexing, masking
+or layout mistake by orders of magnitude.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_25_b200 import binding
+from io_aware_exact_25_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+N_CASES = 24
+
+
+def _check(name, got, ref, wide=False):
+    g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    assert np.all(np.isfinite(g)), f"{name}: non-finite output"
+    err = np.abs(g - ref)
+    _, e = np.frexp(np.abs(ref))
+    bound = np.maximum(2e-2, np.ldexp(1.0, e - 8)) * (2.0 if wide else 1.0)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert np.all(err <= bound), (f"{name}: abs err {err[worst]:.3e} at {worst} (|ref| {abs(ref[worst]):.3e}), "
+                                  f"rel L2 {rel:.3e}")
+    if np.linalg.norm(ref) > 0:
+        assert rel <= 5e-3, f"{name}: rel L2 err {rel:.3e}"
+
+
+def _check_lse(got, ref):
+    g = got.detach().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    empty = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(g), empty), "lse: -inf rows differ"
+    if (~empty).any():
+        assert np.abs(g[~empty] - ref[~empty]).max() <= 1e-3
+
+
+def _draw(case):
+    g = np.random.default_rng(7000 + case)
+    d = int(g.choice([64, 128]))
+    N = int(g.integers(1, 900))
+    B = int(g.integers(1, 3))
+    H = int(g.integers(1, 4))
+    causal = bool(g.integers(0, 2))
+    p = float(g.choice([0.0, 0.0, 0.1, 0.3]))
+    scale = float(g.uniform(0.5, 1.5)) / math.sqrt(d)
+    layout = str(g.choice(["bhsd", "bshd"]))
+    variant = str(g.choice(["plain", "plain", "blocksparse", "splitkv"]))
+    nt = (N + 127) // 128
+    mask = None
+    if variant == "blocksparse":
+        heads = int(g.choice([1, H]))
+        mask = (g.random((heads, nt, nt)) < g.uniform(0.3, 1.0)).astype(np.uint8)
+    splits = int(g.integers(2, 6)) if variant == "splitkv" else 1
+    return dict(B=B, H=H, N=N, d=d, causal=causal, p=p, scale=scale, layout=layout, variant=variant, mask=mask,
+                splits=splits, seed=int(g.integers(0, 2 ** 31)))
+
+
+def _device_view(t, layout, dev):
+    """The same values as a [B,H,N,d] tensor, dense or a view of (B,N,H,d) storage."""
+    if layout == "bhsd":
+        return t.to(dev)
+    return t.transpose(1, 2).contiguous().to(dev).transpose(1, 2)
+
+
+@pytest.mark.parametrize("case", range(N_CASES))
+def test_random_case_matches_oracle(cuda_device, case):
+    c = _draw(case)
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    x = make_inputs(B, H, N, d, seed=c["seed"] % 100000)
+    xd = {n: _device_view(t, c["layout"], cuda_device) for n, t in x.items()}
+    mask = c["mask"]
+    mask_dev = None if mask is None else torch.from_numpy(mask).to(cuda_device)
+    kw = dict(causal=c["causal"], scale=c["scale"], dropout_p=c["p"], seed=c["seed"])
+    if c["variant"] == "splitkv":
+        xc = {n: t.contiguous() for n, t in xd.items()}
+        o, lse = binding.fwd_splitkv(xc["q"], xc["k"], xc["v"], num_splits=c["splits"], **kw)
+        grads = binding.bwd(xc["q"], xc["k"], xc["v"], o, xc["do"], lse, **kw)
+    else:
+        o, lse = binding.fwd(xd["q"], xd["k"], xd["v"], block_mask=mask_dev, **kw)
+        o_l = torch.empty_like(xd["q"])  # the backward reads O in the inputs' layout
+        o_l.copy_(o)
+        grads = binding.bwd(xd["q"], xd["k"], xd["v"], o_l, xd["do"], lse, block_mask=mask_dev, **kw)
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    okw = dict(causal=c["causal"], p_drop=c["p"], seed=c["seed"], block_mask=mask)
+    ro, rlse = oracle.forward(x["q"], x["k"], x["v"], c["scale"], **okw)
+    rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], c["scale"], **okw)
+    rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], c["scale"], **okw)
+    wide = c["scale"] * math.sqrt(d) > 1.0 or c["p"] > 0.1
+    _check("O", o, ro, wide)
+    _check_lse(lse, rlse)
+    if c["p"] > 0 and c["causal"]:
+        # Causal row 0 sees one key, so its exact dQ is 0; the backward forms
+        # D_0 = dO_0 . O_0 from the stored bf16 O_0, and with dropout
+        # O_0 = v_0 / (1 - p) is not a bf16 value.  The rounding leaves
+        # dQ_0 = scale * (dO_0 . (O_0 - bf16(O_0))) * k_0, bounded by
+        # scale * |k_0| * sum |dO_0| * half-ulp(O_0): row 0 is held to that
+        # on top of the absolute bound, the other rows to the full bar.
+        g0 = grads[0][:, :, :1].detach().float().cpu().numpy().reshape(B * H, d)
+        _, eo = np.frexp(np.abs(ro[:, 0]))
+        half_ulp = np.ldexp(1.0, eo - 9)
+        do0 = np.abs(x["do"][:, :, 0].float().numpy().reshape(B * H, d))
+        k0 = np.abs(x["k"][:, :, 0].float().numpy().reshape(B * H, d))
+        bound0 = 2e-2 + c["scale"] * k0 * (do0 * half_ulp).sum(axis=1, keepdims=True)
+        assert np.all(np.abs(g0 - rdq[:, 0]) <= bound0), "dQ row 0 beyond its rounding bound"
+        _check("dQ", grads[0][:, :, 1:], rdq[:, 1:], wide)
+    else:
+        _check("dQ", grads[0], rdq, wide)
+    _check("dK", grads[1], rdk, wide)
+    _check("dV", grads[2], rdv, wide)
+
+
+def test_sweep_covers_every_option():
+    """The drawn cases exercise each option at least once (a guard on the sweep itself)."""
+    cases = [_draw(k) for k in range(N_CASES)]
+    assert {c["d"] for c in cases} == {64, 128}
+    assert {c["causal"] for c in cases} == {False, True}
+    assert {c["layout"] for c in cases} == {"bhsd", "bshd"}
+    assert {c["variant"] for c in cases} == {"plain", "blocksparse", "splitkv"}
+    assert any(c["p"] > 0 for c in cases) and any(c["p"] == 0 for c in cases)
+    assert any(c["N"] % 128 for c in cases)
+    narrow = [c for c in cases if c["scale"] * math.sqrt(c["d"]) <= 1.0 and c["p"] <= 0.1]
+    assert len(narrow) >= N_CASES // 3  # enough cases held to the full bar
