@@ -216,8 +216,8 @@ struct BwdLayout {
   static constexpr uint32_t kOffDQ = (kOffRow + kRowStages * kRowStage + 1023u) & ~1023u;
   static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
-  // row_empty[2], s, dp, p, ds, dv, dk, dq, dq_free, drain
-  static constexpr int kNumBars = 1 + 12 + 9;
+  // row_empty[2], s, dp, p, ds, kv_free, dk, dq, dq_free, drain, acc_free
+  static constexpr int kNumBars = 1 + 12 + 10;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
   // block-sparse: the query-tile bit set and its count after the barriers
   static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
@@ -258,27 +258,41 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* bar_dp = bars + 14;
   uint64_t* bar_p = bars + 15;
   uint64_t* bar_ds = bars + 16;
-  uint64_t* bar_dv = bars + 17;
+  uint64_t* bar_kv_free = bars + 17;  // K/V buffers no longer read (last MMA of an item)
   uint64_t* bar_dk = bars + 18;
   uint64_t* bar_dq = bars + 19;
   uint64_t* bar_dq_free = bars + 20;
   uint64_t* bar_drain = bars + 21;
+  uint64_t* bar_acc_free = bars + 22;  // dV/dK accumulators read out by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);  // [0] abort, [1] dQ warpgroup flag
   const uint32_t sbase = smem_u32(smem);
 
   const int BH = a.B * a.H;
   const int nT = (a.N + 127) >> 7;
-  // CTA order: key tiles ascending (the most query tiles first when causal:
-  // longest-processing-time order), heads interleaved.  The CTAs of a wave
-  // sweep the query tiles of their heads in near lockstep, so the Q/dO tiles
-  // and accumulator rows they share stay in L2.
-  const int jt = blockIdx.x / BH;  // key tile
-  const int bh = blockIdx.x - jt * BH;
-  const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
-  const int i_begin = CAUSAL ? jt : 0;
-  int n_steps = nT - i_begin;  // query tiles this CTA visits
   const int npad = nT * 128;
+  // Work items (key tile, head) in longest-processing-time order: key tiles
+  // ascending (the most query tiles first when causal), heads interleaved, so
+  // the CTAs working at one time sweep the query tiles of their heads in near
+  // lockstep and the Q/dO tiles and accumulator rows they share stay in L2.
+  // The grid is persistent: each CTA takes one item per round (see
+  // item_index); the next item's first products overlap the last item's dQ
+  // reductions and dK/dV write-out.  (Block-sparse kernels run one item per
+  // CTA.)
+  const int n_items = BH * nT;
+  struct Item {
+    int jt, bh, bb, hh, i_begin, n_steps;
+  };
+  auto item_of = [&](int w) {
+    Item t;
+    t.jt = w / BH;
+    t.bh = w - t.jt * BH;
+    t.bb = t.bh / a.H;
+    t.hh = t.bh - t.bb * a.H;
+    t.i_begin = CAUSAL ? t.jt : 0;
+    t.n_steps = nT - t.i_begin;
+    return t;
+  };
   uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // SPARSE: query tiles that see jt
   int* sparse_cnt = reinterpret_cast<int*>(qbits + kSparseWords);
   const int nwords = (nT + 31) >> 5;
@@ -297,7 +311,8 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
     mbar_init(bar_ds, 256);
-    mbar_init(bar_dv, 1);
+    mbar_init(bar_kv_free, 1);
+    mbar_init(bar_acc_free, 256);
     mbar_init(bar_dk, 1);
     mbar_init(bar_dq, 1);
     mbar_init(bar_dq_free, 128);
@@ -313,9 +328,10 @@ __global__ void __launch_bounds__(448, 1)
   }
   if (SPARSE && warp == 13) {
     // column jt of the mask: entry (i, jt) for i in [i_begin, nT)
-    const int hm = a.bmask_heads == 1 ? 0 : hh;
-    const uint8_t* col = a.bmask + (size_t)hm * nT * nT + jt;
-    const int3 c = build_bit_sets(col, nT, nullptr, 0, i_begin, nT, nwords, qbits, nullptr, lane);
+    const Item t = item_of(blockIdx.x);
+    const int hm = a.bmask_heads == 1 ? 0 : t.hh;
+    const uint8_t* col = a.bmask + (size_t)hm * nT * nT + t.jt;
+    const int3 c = build_bit_sets(col, nT, nullptr, 0, t.i_begin, nT, nwords, qbits, nullptr, lane);
     if (lane == 0) sparse_cnt[0] = c.x;
   }
   tc_fence_before();
@@ -324,71 +340,111 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, a.err};
   const bool run = *abort_flag == 0;
-  if (SPARSE) n_steps = sparse_cnt[0];
+  // Item of round r for this CTA: rounds alternate direction across the grid
+  // ("snake" order), so with items sorted by decreasing length every CTA gets
+  // nearly the same total work.
+  auto item_index = [&](int r) {
+    const int G = (int)gridDim.x, c = (int)blockIdx.x;
+    return r * G + ((r & 1) ? (G - 1 - c) : c);
+  };
+  // the items of this CTA, with the block-sparse step count
+  auto item_at = [&](int w) {
+    Item t = item_of(w);
+    if (SPARSE) t.n_steps = sparse_cnt[0];
+    return t;
+  };
 
   if (run && warp == 13) {
     // ------------------------------------------------------ TMA producer
     const uint64_t pol_keep = policy_evict_last();
-    if (lane == 0 && n_steps > 0) {  // (a key tile no query tile sees loads nothing)
+    if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
-      mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, jt * 128, hh, bb, bar_kv, pol_keep);
-        tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, jt * 128, hh, bb, bar_kv, pol_keep);
-      }
     }
-    // All 32 lanes run this loop (they compute the dropout row keys); the
+    // All 32 lanes run these loops (they compute the dropout row keys); the
     // waits are made warp-uniform with __all_sync, lane 0 issues the copies.
-    int q_issued = 0, do_issued = 0;
+    // g counts query-tile steps over all items of the CTA and drives the
+    // rings' stages and phases.
+    int q_issued = 0, do_issued = 0, kv_issued = 0;
+    int g = 0;
     bool ok = true;
-    BitWalk walk(qbits, qbits, nwords);
-    for (int it = 0; it < n_steps && ok; ++it) {
-      const int i = SPARSE ? walk.next() : i_begin + it;
-      // Q_i and dO_i: re-read by every key tile of the head -> keep in L2
-      const int qs = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_q_empty[qs], ((it >> 1) & 1) ^ 1u, ab))) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, hh, bb,
-                      &bar_q_full[qs], pol_keep);
-      }
-      ++q_issued;
-      const int ds_ = it % L::kDoStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_do_empty[ds_], ((it / L::kDoStages) & 1) ^ 1u, ab))) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_do_full[ds_], L::kTile);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, hh, bb,
-                      &bar_do_full[ds_], pol_keep);
-      }
-      ++do_issued;
-      // row statistics of query tile i
-      const int rs = it % L::kRowStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_row_empty[rs], ((it / L::kRowStages) & 1) ^ 1u, ab))) {
-        ok = false;
-        break;
-      }
-      uint8_t* rowbuf = smem + L::kOffRow + rs * L::kRowStage;
-      if (DROPOUT) {
-        uint32_t* keys = reinterpret_cast<uint32_t*>(rowbuf + 2 * 512);
-        for (int c = lane; c < 128; c += 32)
-          keys[c] = dropout_row_key(a.seed, (uint32_t)bb, (uint32_t)hh, (uint32_t)(i * 128 + c));
+    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+      const int w = item_index(r);
+      if (w >= n_items) continue;
+      const Item t = item_at(w);
+      if (t.n_steps == 0) continue;  // (a key tile no query tile sees loads nothing)
+      BitWalk walk(qbits, qbits, nwords);
+      for (int it = 0; it < t.n_steps; ++it) {
+        const int gs = g + it;
+        const int i = SPARSE ? walk.next() : t.i_begin + it;
+        // Q_i and dO_i: re-read by every key tile of the head -> keep in L2
+        const int qs = gs & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_q_empty[qs], ((gs >> 1) & 1) ^ 1u, ab))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, t.hh, t.bb,
+                        &bar_q_full[qs], pol_keep);
+        }
+        ++q_issued;
+        const int ds_ = gs % L::kDoStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_do_empty[ds_], ((gs / L::kDoStages) & 1) ^ 1u, ab))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_do_full[ds_], L::kTile);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, t.hh, t.bb,
+                        &bar_do_full[ds_], pol_keep);
+        }
+        ++do_issued;
+        // row statistics of query tile i
+        const int rs = gs % L::kRowStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_row_empty[rs], ((gs / L::kRowStages) & 1) ^ 1u, ab))) {
+          ok = false;
+          break;
+        }
+        uint8_t* rowbuf = smem + L::kOffRow + rs * L::kRowStage;
+        if (DROPOUT) {
+          uint32_t* keys = reinterpret_cast<uint32_t*>(rowbuf + 2 * 512);
+          for (int c = lane; c < 128; c += 32)
+            keys[c] = dropout_row_key(a.seed, (uint32_t)t.bb, (uint32_t)t.hh, (uint32_t)(i * 128 + c));
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_row_full[rs], 1024);
+          bulk_load(rowbuf, a.lse2 + (size_t)t.bh * npad + i * 128, 512, &bar_row_full[rs]);
+          bulk_load(rowbuf + 512, a.drow + (size_t)t.bh * npad + i * 128, 512, &bar_row_full[rs]);
+        }
         __syncwarp();
+        if (it == 0) {
+          // K_j, V_j, after the item's first Q/dO/row loads (which only need
+          // ring slots): the previous item's last product must have read them
+          if (kv_issued > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_kv_free, (kv_issued - 1) & 1, ab))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
+            for (int h = 0; h < D / 64; ++h) {
+              tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
+              tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
+            }
+          }
+          ++kv_issued;
+        }
       }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_row_full[rs], 1024);
-        bulk_load(rowbuf, a.lse2 + (size_t)bh * npad + i * 128, 512, &bar_row_full[rs]);
-        bulk_load(rowbuf + 512, a.drow + (size_t)bh * npad + i * 128, 512, &bar_row_full[rs]);
-      }
-      __syncwarp();
+      g += t.n_steps;
     }
-    if (lane == 0 && n_steps > 0) {
+    if (lane == 0) {
       // Every load issued must land before the CTA may exit.
-      mbar_wait_drain(bar_kv, 0);
+      if (kv_issued > 0) mbar_wait_drain(bar_kv, (kv_issued - 1) & 1);
       for (int n = q_issued > 2 ? q_issued - 2 : 0; n < q_issued; ++n) mbar_wait_drain(&bar_q_full[n & 1], (n >> 1) & 1);
       for (int n = do_issued > L::kDoStages ? do_issued - L::kDoStages : 0; n < do_issued; ++n)
         mbar_wait_drain(&bar_do_full[n % L::kDoStages], (n / L::kDoStages) & 1);
@@ -400,18 +456,9 @@ __global__ void __launch_bounds__(448, 1)
       constexpr uint32_t kIdTM = idesc_bf16(128, D, false, true);     // dV, dK: A K-major, B MN-major
       constexpr uint32_t kIdMM = idesc_bf16(128, D, true, true);      // dQ: both MN-major
       const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sDS = sbase + L::kOffDS;
-      bool ok = n_steps > 0 && mbar_wait(bar_kv, 0, ab) && mbar_wait(&bar_q_full[0], 0, ab);
+      bool ok = true;
       bool issued_any = false;
-      if (ok) {
-        tc_fence_after();
-        const uint32_t sQ0 = sbase + L::kOffQ;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQ0, kk, L::kHalf), kIdKK,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar_s);
-        issued_any = true;
-      }
+      int g = 0, kv_used = 0;
       // Per step: dP(i), dV(i), S(i+1), dQ(i), dK(i).  dP(i) overwrites the
       // dQ(i-1) partial and waits for the dQ warpgroup to have read it; it then
       // runs while the softmax warps form P(i).  S(i+1) overwrites the columns
@@ -421,57 +468,94 @@ __global__ void __launch_bounds__(448, 1)
       // warps form dS(i), and P(i+1) can start as soon as dS(i) is done.  dQ(i)
       // and dK(i) both read dS from shared memory (dS^T for dK is the same tile
       // read K-major); dQ(i) goes first so its read-out, which gates dP(i+1),
-      // starts while dK(i) runs.
-      for (int it = 0; it < n_steps && ok; ++it) {
-        const uint32_t ph = it & 1;
-        const int qs = it & 1;
-        const int ds_ = it % L::kDoStages;
-        const uint32_t sQ = sbase + L::kOffQ + qs * L::kTile;
-        const uint32_t sDO = sbase + L::kOffDO + ds_ * L::kTile;
-        // dP^T = V dO_i^T into R_dP
-        if (!mbar_wait(&bar_do_full[ds_], (it / L::kDoStages) & 1, ab)) break;
-        if (it > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab)) break;
+      // starts while dK(i) runs.  Across items the same order holds: the next
+      // item's S(0) is queued behind the last dK, its first dV and dK (which
+      // overwrite the accumulators) wait for the epilogue to have read them.
+      for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+      const int w = item_index(r);
+      if (w >= n_items) continue;
+        const Item t = item_at(w);
+        if (t.n_steps == 0) continue;
+        ok = mbar_wait(bar_kv, kv_used & 1, ab) && mbar_wait(&bar_q_full[g & 1], (g >> 1) & 1, ab);
+        if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + L::kColDP, desc_kmajor(sV, kk, L::kHalf), desc_kmajor(sDO, kk, L::kHalf), kIdKK,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar_dp);
-        // dV += P^T dO_i
-        if (!mbar_wait(bar_p, ph, ab)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::kColDV, tmem + L::kColS + packed_col(kk), desc_mnmajor(sDO, kk, L::kHalf), kIdTM,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar_do_empty[ds_]);
-        // S^T for the next step (behind dV, which reads P^T from R_S)
-        if (it + 1 < n_steps) {
-          const int qn = (it + 1) & 1;
-          if (!mbar_wait(&bar_q_full[qn], ((it + 1) >> 1) & 1, ab)) break;
-          tc_fence_after();
-          const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
+        {
+          const uint32_t sQ0 = sbase + L::kOffQ + (g & 1) * L::kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQn, kk, L::kHalf), kIdKK,
+            mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQ0, kk, L::kHalf), kIdKK,
                    kk > 0 ? 1u : 0u);
           mma_commit(bar_s);
+          issued_any = true;
         }
-        // dQ_i partial = dS K_j into R_dP (the softmax warps have read dP^T(i))
-        if (!mbar_wait(bar_ds, ph, ab)) break;
-        tc_fence_after();
+        for (int it = 0; it < t.n_steps && ok; ++it) {
+          const int gs = g + it;
+          const uint32_t ph = gs & 1;
+          const int qs = gs & 1;
+          const int ds_ = gs % L::kDoStages;
+          const uint32_t sQ = sbase + L::kOffQ + qs * L::kTile;
+          const uint32_t sDO = sbase + L::kOffDO + ds_ * L::kTile;
+          // dP^T = V dO_i^T into R_dP
+          if (!mbar_wait(&bar_do_full[ds_], (gs / L::kDoStages) & 1, ab) ||
+              (gs > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);
-        // dK += dS^T Q_i, A = the shared dS tile read K-major (rows = keys)
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + L::kColDP, desc_kmajor(sV, kk, L::kHalf), desc_kmajor(sDO, kk, L::kHalf), kIdKK,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_dp);
+          // dV += P^T dO_i; the item's first one overwrites the accumulator
+          if (!mbar_wait(bar_p, ph, ab) || (it == 0 && kv_used > 0 && !mbar_wait(bar_acc_free, (kv_used - 1) & 1, ab))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::kColDK, desc_kmajor(sDS, kk, L::kHalf), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_dk);
-        mma_commit(&bar_q_empty[qs]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::kColDV, tmem + L::kColS + packed_col(kk), desc_mnmajor(sDO, kk, L::kHalf), kIdTM,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar_do_empty[ds_]);
+          // S^T for the next step (behind dV, which reads P^T from R_S)
+          if (it + 1 < t.n_steps) {
+            const int qn = (gs + 1) & 1;
+            if (!mbar_wait(&bar_q_full[qn], ((gs + 1) >> 1) & 1, ab)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sQn = sbase + L::kOffQ + qn * L::kTile;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + L::kColS, desc_kmajor(sK, kk, L::kHalf), desc_kmajor(sQn, kk, L::kHalf), kIdKK,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(bar_s);
+          }
+          // dQ_i partial = dS K_j into R_dP (the softmax warps have read dP^T(i))
+          if (!mbar_wait(bar_ds, ph, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_dq);
+          // dK += dS^T Q_i, A = the shared dS tile read K-major (rows = keys)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + L::kColDK, desc_kmajor(sDS, kk, L::kHalf), desc_mnmajor(sQ, kk, L::kHalf), kIdTM,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_dk);
+          mma_commit(&bar_q_empty[qs]);
+        }
+        if (!ok) break;
+        mma_commit(bar_kv_free);  // the item's products have read K_j and V_j
+        ++kv_used;
+        g += t.n_steps;
       }
       if (issued_any) {
         mma_commit(bar_drain);
@@ -515,18 +599,27 @@ __global__ void __launch_bounds__(448, 1)
         bulk_commit();
       }
     };
+    int g = 0;
+    bool ok = true;
+    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+      const int w = item_index(r);
+      if (w >= n_items) continue;
+    const Item t = item_at(w);
     BitWalk walk(qbits, qbits, nwords);
-    for (int it = 0; it < n_steps; ++it) {
-      const int i = SPARSE ? walk.next() : i_begin + it;
+    for (int it = 0; it < t.n_steps; ++it) {
+      const int i = SPARSE ? walk.next() : t.i_begin + it;
       // the staging tiles are free once the previous step's reductions read them
       if (leader) {
         bulk_wait_read<0>();
-        *dq_flag = mbar_wait(bar_dq, it & 1, ab) ? 1 : 0;
+        *dq_flag = mbar_wait(bar_dq, (g + it) & 1, ab) ? 1 : 0;
       }
       named_bar_sync(1, 128);
-      if (*dq_flag == 0) break;
+      if (*dq_flag == 0) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      float* acc_tile = a.dq_acc + ((size_t)bh * nT + i) * (size_t)(128 * D);
+      float* acc_tile = a.dq_acc + ((size_t)t.bh * nT + i) * (size_t)(128 * D);
       if (D == 64) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tQ, v0);
@@ -572,13 +665,14 @@ __global__ void __launch_bounds__(448, 1)
         reduce(acc_tile, 4, 4);
       }
     }
+    g += t.n_steps;
+    }
     if (leader) bulk_wait_all();
   } else if (run && warp < 8) {
     // --------------------------------------------------------- P and dS
     const int wg = warp >> 2;
     const int quad = warp & 3;
     const int jr = quad * 32 + lane;  // key within the tile == TMEM lane
-    const int key = jt * 128 + jr;
     const int col0 = 64 * wg;         // this warpgroup's query columns
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + L::kColS + col0;
@@ -586,15 +680,23 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t tPst = tmem + lane_off + L::kColS + 64u * wg;   // packed P^T (32 columns)
     const uint32_t sDSrow = sbase + L::kOffDS + wg * L::kHalf + jr * 128;
     const float sl2 = a.scale_log2;
-    const bool key_ok = key < a.N;
     bool ok = true;
+    int g = 0;
+    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+      const int w = item_index(r);
+      if (w >= n_items) continue;
+    const Item t = item_at(w);
+    const int jt = t.jt, bb = t.bb, hh = t.hh;
+    const int key = jt * 128 + jr;
+    const bool key_ok = key < a.N;
     BitWalk walk(qbits, qbits, nwords);
-    for (int it = 0; it < n_steps; ++it) {
-      const int i = SPARSE ? walk.next() : i_begin + it;
-      const uint32_t ph = it & 1;
-      const int rs = it % L::kRowStages;
+    for (int it = 0; it < t.n_steps; ++it) {
+      const int i = SPARSE ? walk.next() : t.i_begin + it;
+      const int gs = g + it;
+      const uint32_t ph = gs & 1;
+      const int rs = gs % L::kRowStages;
       const uint32_t rowbuf = sbase + L::kOffRow + rs * L::kRowStage;
-      if (!mbar_wait(bar_s, ph, ab) || !mbar_wait(&bar_row_full[rs], (it / L::kRowStages) & 1, ab)) {
+      if (!mbar_wait(bar_s, ph, ab) || !mbar_wait(&bar_row_full[rs], (gs / L::kRowStages) & 1, ab)) {
         ok = false;
         break;
       }
@@ -685,7 +787,7 @@ __global__ void __launch_bounds__(448, 1)
         break;
       }
       // dQ(i-1) and dK(i-1) read sDS; wait for the later one before overwriting
-      if (it > 0 && !mbar_wait(bar_dk, ph ^ 1u, ab)) {
+      if (gs > 0 && !mbar_wait(bar_dk, ph ^ 1u, ab)) {
         ok = false;
         break;
       }
@@ -734,8 +836,10 @@ __global__ void __launch_bounds__(448, 1)
       mbar_arrive(bar_ds);
       mbar_arrive(&bar_row_empty[rs]);
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK = scale * acc
-    if (SPARSE && n_steps == 0) {
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK = scale * acc,
+    // then both release the accumulators to the next item's first products
+    if (!ok) break;
+    if (SPARSE && t.n_steps == 0) {
       // no query tile sees this key tile
       __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + (long long)key * a.dv_sn
                                    : a.dk + bb * a.dk_sb + hh * a.dk_sh + (long long)key * a.dk_sn;
@@ -743,7 +847,11 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int c = 0; c < D; c += 8) st_global_v4(dst + c, 0u, 0u, 0u, 0u);
       }
-    } else if (ok && n_steps > 0 && mbar_wait(bar_dk, (n_steps - 1) & 1, ab)) {
+    } else if (t.n_steps > 0) {
+      if (!mbar_wait(bar_dk, (g + t.n_steps - 1) & 1, ab)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
       const float mul = wg == 0 ? 1.f : a.scale;
@@ -763,6 +871,10 @@ __global__ void __launch_bounds__(448, 1)
             st_global_v4(dst + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar_acc_free);
+    }
+    g += t.n_steps;
     }
   }
 
@@ -782,7 +894,14 @@ cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const 
   const int smem = (int)(SPARSE ? L::kSmemSparse : L::kSmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
+  // one CTA per SM looping over the work items (block-sparse: one CTA per item)
+  long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
+  if (!SPARSE) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0 && grid > sms)
+      grid = sms;
+  }
   kern<<<(unsigned)grid, L::kThreads, smem, st>>>(mq, mk, mv, mdo, a);
   return cudaGetLastError();
 }
