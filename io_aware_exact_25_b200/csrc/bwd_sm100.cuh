@@ -343,7 +343,12 @@ __global__ void __launch_bounds__(448, 1)
   // Item of round r for this CTA: rounds alternate direction across the grid
   // ("snake" order), so with items sorted by decreasing length every CTA gets
   // nearly the same total work.
+  // Dropout and block-sparse kernels run one item per CTA (see the launch);
+  // for them the loops below make a single pass that the compiler folds.
+  constexpr bool PERSIST = !SPARSE && !DROPOUT;
+  const int n_rounds = PERSIST ? (n_items + (int)gridDim.x - 1) / (int)gridDim.x : 1;
   auto item_index = [&](int r) {
+    if (!PERSIST) return (int)blockIdx.x;
     const int G = (int)gridDim.x, c = (int)blockIdx.x;
     return r * G + ((r & 1) ? (G - 1 - c) : c);
   };
@@ -370,11 +375,22 @@ __global__ void __launch_bounds__(448, 1)
     int q_issued = 0, do_issued = 0, kv_issued = 0;
     int g = 0;
     bool ok = true;
-    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+    for (int r = 0; r < n_rounds && ok; ++r) {
       const int w = item_index(r);
       if (w >= n_items) continue;
       const Item t = item_at(w);
       if (t.n_steps == 0) continue;  // (a key tile no query tile sees loads nothing)
+      auto load_kv = [&]() {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
+          for (int h = 0; h < D / 64; ++h) {
+            tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
+            tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
+          }
+        }
+        ++kv_issued;
+      };
+      if (!PERSIST) load_kv();  // one item per CTA: K/V first
       BitWalk walk(qbits, qbits, nwords);
       for (int it = 0; it < t.n_steps; ++it) {
         const int gs = g + it;
@@ -423,21 +439,14 @@ __global__ void __launch_bounds__(448, 1)
           bulk_load(rowbuf + 512, a.drow + (size_t)t.bh * npad + i * 128, 512, &bar_row_full[rs]);
         }
         __syncwarp();
-        if (it == 0) {
+        if (PERSIST && it == 0) {
           // K_j, V_j, after the item's first Q/dO/row loads (which only need
           // ring slots): the previous item's last product must have read them
           if (kv_issued > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_kv_free, (kv_issued - 1) & 1, ab))) {
             ok = false;
             break;
           }
-          if (lane == 0) {
-            mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
-            for (int h = 0; h < D / 64; ++h) {
-              tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
-              tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
-            }
-          }
-          ++kv_issued;
+          load_kv();
         }
       }
       g += t.n_steps;
@@ -471,7 +480,7 @@ __global__ void __launch_bounds__(448, 1)
       // starts while dK(i) runs.  Across items the same order holds: the next
       // item's S(0) is queued behind the last dK, its first dV and dK (which
       // overwrite the accumulators) wait for the epilogue to have read them.
-      for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+      for (int r = 0; r < n_rounds && ok; ++r) {
       const int w = item_index(r);
       if (w >= n_items) continue;
         const Item t = item_at(w);
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(448, 1)
     };
     int g = 0;
     bool ok = true;
-    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+    for (int r = 0; r < n_rounds && ok; ++r) {
       const int w = item_index(r);
       if (w >= n_items) continue;
     const Item t = item_at(w);
@@ -682,7 +691,7 @@ __global__ void __launch_bounds__(448, 1)
     const float sl2 = a.scale_log2;
     bool ok = true;
     int g = 0;
-    for (int r = 0; r * (int)gridDim.x < n_items && ok; ++r) {
+    for (int r = 0; r < n_rounds && ok; ++r) {
       const int w = item_index(r);
       if (w >= n_items) continue;
     const Item t = item_at(w);
@@ -894,9 +903,12 @@ cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const 
   const int smem = (int)(SPARSE ? L::kSmemSparse : L::kSmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  // one CTA per SM looping over the work items (block-sparse: one CTA per item)
+  // One CTA per SM looping over the work items.  Block-sparse and dropout
+  // kernels run one CTA per item: block-sparse items differ in length in ways
+  // only the mask knows, and with dropout (one row-statistics stage at
+  // d = 128) the persistent grid measured 10% slower on N = 65536.
   long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
-  if (!SPARSE) {
+  if (!SPARSE && !DROPOUT) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0 && grid > sms)
