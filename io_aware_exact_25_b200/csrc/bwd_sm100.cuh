@@ -39,8 +39,9 @@
 //   warp  12    tcgen05 MMA issue (one thread)
 //   warp  13    TMA producer (+ dropout row keys)
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
-// [0,32) and [64,96); R_dP [128,256) dP^T fp32, then the dQ partial (fp32,
-// D columns); dV at 256, dK at 256 + D.  dS goes to shared memory only.  MMA
+// [0,32) and [64,96); R_dP [128,256) dP^T fp32, then (d = 128) the dQ
+// partial (fp32, D columns); dV at 256, dK at 256 + D; at d = 64 the dQ
+// partial has its own columns at 384.  dS goes to shared memory only.  MMA
 // order per step: dP(i), dV(i), S(i+1), dQ(i), dK(i); dP(i) runs while the
 // softmax warps form P(i), S(i+1) while they form dS(i), and the dQ read-out
 // of one step overlaps dK and the next step's P.
@@ -225,6 +226,10 @@ struct BwdLayout {
   static_assert(kOffDQ % 1024 == 0, "staging tiles must be swizzle-aligned");
   static_assert(kSmemSparse <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  // d = 64 leaves 128 columns free: the dQ partial gets its own, so dP(i+1)
+  // need not wait for the dQ(i) read-out; at d = 128 it shares dP's columns
+  static constexpr bool kOwnDQ = D == 64;
+  static constexpr uint32_t kColDQ = kOwnDQ ? 256 + 2 * D : kColDP;
 };
 
 // TMEM column of the packed bf16 P^T slice kk (16 queries) written by the
@@ -468,9 +473,10 @@ __global__ void __launch_bounds__(448, 1)
       bool ok = true;
       bool issued_any = false;
       int g = 0, kv_used = 0;
-      // Per step: dP(i), dV(i), S(i+1), dQ(i), dK(i).  dP(i) overwrites the
-      // dQ(i-1) partial and waits for the dQ warpgroup to have read it; it then
-      // runs while the softmax warps form P(i).  S(i+1) overwrites the columns
+      // Per step: dP(i), dV(i), S(i+1), dQ(i), dK(i).  At d = 128 dP(i)
+      // overwrites the dQ(i-1) partial and waits for the dQ warpgroup to have
+      // read it (at d = 64 dQ(i) waits instead); dP(i) then runs while the
+      // softmax warps form P(i).  S(i+1) overwrites the columns
       // holding P^T(i), which dV(i) reads; it is queued behind its reader and
       // the tensor core executes one thread's MMAs in order, so it needs no
       // wait.  S(i+1) goes right behind dV(i) so it runs while the softmax
@@ -506,7 +512,7 @@ __global__ void __launch_bounds__(448, 1)
           const uint32_t sDO = sbase + L::kOffDO + ds_ * L::kTile;
           // dP^T = V dO_i^T into R_dP
           if (!mbar_wait(&bar_do_full[ds_], (gs / L::kDoStages) & 1, ab) ||
-              (gs > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab))) {
+              (!L::kOwnDQ && gs > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab))) {
             ok = false;
             break;
           }
@@ -542,15 +548,16 @@ __global__ void __launch_bounds__(448, 1)
                      kk > 0 ? 1u : 0u);
             mma_commit(bar_s);
           }
-          // dQ_i partial = dS K_j into R_dP (the softmax warps have read dP^T(i))
-          if (!mbar_wait(bar_ds, ph, ab)) {
+          // dQ_i partial = dS K_j (the softmax warps have read dP^T(i)); with
+          // its own columns it waits for the previous partial's read-out here
+          if (!mbar_wait(bar_ds, ph, ab) || (L::kOwnDQ && gs > 0 && !mbar_wait(bar_dq_free, ph ^ 1u, ab))) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + L::kColDP, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
+            mma_ss(tmem + L::kColDQ, desc_mnmajor(sDS, kk, L::kHalf), desc_mnmajor(sK, kk, L::kHalf), kIdMM,
                    kk > 0 ? 1u : 0u);
           mma_commit(bar_dq);
           // dK += dS^T Q_i, A = the shared dS tile read K-major (rows = keys)
@@ -586,7 +593,7 @@ __global__ void __launch_bounds__(448, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query within the tile == TMEM lane
     const bool leader = warp == 8 && lane == 0;
-    const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDP;
+    const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDQ;
     const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
     volatile int* dq_flag = abort_flag + 1;
     // stage 32 columns (two 16-column pieces) of this row into tiles t, t+1
