@@ -239,6 +239,19 @@ int fa_bwd_recompute_blocksparse(const void* q, const void* k, const void* v, co
 int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,
                     const int32_t* rows, int nrows, uint8_t* out, void* stream);
 
+/*
+ * Fault injection for tests (the paper has no counterpart): fa_fwd on dense
+ * tensors with the producer warp issuing no K/V load, so the MMA warp's first
+ * bounded wait runs out (after about 2 s).  The kernel then records code 1
+ * (timeout) in the device error word, every warp leaves its loop, tensor
+ * memory is freed and the kernel exits; o and lse are left unwritten.  The
+ * call itself returns the launch status (FA_OK); fa_get_device_error reports
+ * the timeout and clears it, and the context stays usable.  No fault, trap or
+ * hang is involved.
+ */
+int fa_debug_fwd_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                         int d, float scale, int causal, void* stream);
+
 /* Static description of a status code. */
 const char* fa_strerror(int status);
 

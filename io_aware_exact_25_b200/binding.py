@@ -30,7 +30,7 @@ FA_ERR_TOO_LARGE = -7
 EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
-           "fa_bwd_recompute_blocksparse",
+           "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout",
            "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -78,6 +78,7 @@ def load() -> ctypes.CDLL:
                                            vp, SZ, vp]
         lib.fa_bwd_recompute_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, I, vp, SZ,
                                                      vp]
+        lib.fa_debug_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
         lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
@@ -91,6 +92,7 @@ def load() -> ctypes.CDLL:
         for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
                    lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
                    lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
+                   lib.fa_debug_fwd_timeout,
                    lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
@@ -304,6 +306,21 @@ def dropout_mask(B, H, N, dropout_p, seed, heads, rows, device="cuda", stream=No
                                 r.numel(), _ptr(out), _stream(stream))
     _call(rc, "fa_dropout_mask")
     return out
+
+
+def debug_fwd_timeout(q, k, v, causal=False, scale=None, stream=None) -> int:
+    """Run ``fa_debug_fwd_timeout`` (fault injection: a forward whose first
+    bounded wait runs out); returns the launch status.  Read the outcome with
+    ``device_error``."""
+    _check_inputs(q, k, v)
+    _check_dense(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    return int(load().fa_debug_fwd_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                           int(bool(causal)), _stream(stream)))
 
 
 def device_error(stream=None) -> int:

@@ -203,7 +203,8 @@ namespace {
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides, int B,
              int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int num_splits,
-             void* workspace, size_t workspace_bytes, const uint8_t* bmask, int bmask_heads, void* stream) {
+             void* workspace, size_t workspace_bytes, const uint8_t* bmask, int bmask_heads, void* stream,
+             int debug_skip_kv = 0) {
   int rc = check_common(B, H, N, d, scale, causal, dropout_p);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -240,6 +241,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   a.part_lse = nullptr;
   a.bmask = bmask;
   a.bmask_heads = bmask_heads;
+  a.debug_skip_kv = debug_skip_kv;
   if (num_splits > 1) {
     a.part_o = static_cast<float*>(workspace);
     a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -302,6 +304,13 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const fa_strides s = contiguous_strides(H, N, d);
   const fa_strides all[4] = {s, s, s, s};
   return fa_fwd_strided(q, k, v, o, lse, all, B, H, N, d, scale, causal, dropout_p, seed, stream);
+}
+
+int fa_debug_fwd_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                         int d, float scale, int causal, void* stream) {
+  const fa_strides s = contiguous_strides(H, N, d);
+  const fa_strides all[4] = {s, s, s, s};
+  return fwd_impl(q, k, v, o, lse, all, B, H, N, d, scale, causal, 0.f, 0, 1, nullptr, 0, nullptr, 0, stream, 1);
 }
 
 int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,

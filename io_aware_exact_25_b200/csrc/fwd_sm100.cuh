@@ -62,6 +62,9 @@ struct FwdArgs {
   // tile qt see key tile kt; hm = 0 when bmask_heads == 1, else the head
   const uint8_t* bmask;
   int bmask_heads;
+  // fault injection for tests: the producer issues no K/V load, so the MMA
+  // warp's first wait runs out and the kernel reports a timeout
+  int debug_skip_kv;
 };
 
 // Kernel variants: plain, split-KV, block-sparse.
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(320, 1)
       int issued = 0;
       bool ok = true;
       BitWalk walk(bits0, bits1, nwords);
-      for (int j = 0; j < nkv_max && ok; ++j) {
+      for (int j = 0; j < nkv_max && ok && !a.debug_skip_kv; ++j) {
         const int kt = SPARSE ? walk.next() : j0 + j;  // key tile of this step
         for (int which = 0; which < 2; ++which) {
           if (!mbar_wait(&bar_kv_empty[stage], phase ^ 1u, ab)) {
