@@ -133,8 +133,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * [B,H,N,d] bf16.  workspace (16-byte aligned, at least
  * fa_bwd_workspace_size bytes) is scratch owned by the caller; its contents
  * on entry do not matter.  dq/dk/dv must not alias any input.
- * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.  dQ is accumulated in fp32 with atomic adds, so its bits may differ from run
- * to run by rounding order; dK and dV are deterministic.
+ * Errors: as fa_fwd, plus FA_ERR_WORKSPACE.  dQ: each key tile's partial
+ * dQ_i = dS K_j is staged in shared memory and added into an fp32 workspace
+ * accumulator with bulk reductions (cp.reduce.async.bulk .add.f32); the order
+ * of those additions varies, so dq bits may differ from run to run by
+ * rounding; dk and dv are deterministic.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, float dropout_p,

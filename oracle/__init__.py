@@ -77,6 +77,8 @@ def _load():
         lib.orc_num_threads.restype = ctypes.c_int
         lib.orc_set_block_mask.argtypes = [u8p, I, I]
         lib.orc_set_block_mask.restype = None
+        lib.orc_set_seqlens.argtypes = [i32p]
+        lib.orc_set_seqlens.restype = None
         _lib = lib
         return lib
 
@@ -123,6 +125,33 @@ def _p(a, ctype):
     return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctype))
 
 
+class _SeqLens:
+    """Installs per-batch sequence lengths for the oracle calls made inside
+    the ``with``: rows and keys at or beyond ``seqlens[b]`` of batch entry b
+    are padding ("FlashAttention for Efficient Training", section 5.2:
+    A_ij = -inf unless the key lies within the sequence).  Padding queries
+    get O = 0, lse = -inf and dQ = 0; padding keys get dK = dV = 0."""
+
+    def __init__(self, seqlens, B, N):
+        self.arr = None
+        if seqlens is None:
+            return
+        a = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int64))
+        if a.shape != (B,) or (a < 0).any() or (a > N).any():
+            raise ValueError(f"seqlens must be {B} lengths in [0, {N}], got {a.tolist()}")
+        self.arr = a.astype(np.int32)
+
+    def __enter__(self):
+        if self.arr is not None:
+            _load().orc_set_seqlens(_p(self.arr, ctypes.c_int32))
+        return self
+
+    def __exit__(self, *exc):
+        if self.arr is not None:
+            _load().orc_set_seqlens(None)
+        return False
+
+
 class _BlockMask:
     """Installs a block mask for the oracle calls made inside the ``with``.
 
@@ -161,13 +190,14 @@ def num_threads() -> int:
 
 
 def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None,
-            block_mask=None, block=128):
+            block_mask=None, block=128, seqlens=None):
     """O_i and lse_i for the selected heads (bh = b*H + h) and query rows.
 
     Returns ``(o, lse)`` as float64 arrays of shape ``[nheads, nrows, d]`` and
     ``[nheads, nrows]``.  ``block_mask`` (``[1 or H, nt, nt]`` over
     ``block``-sized tiles) hides whole key tiles; a row that sees no key gets
-    O = 0 and lse = -inf.
+    O = 0 and lse = -inf.  ``seqlens`` (``[B]``) marks rows and keys at or
+    beyond ``seqlens[b]`` of batch entry b as padding.
     """
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     f64 = _kind(qb, kb, vb)
@@ -176,7 +206,7 @@ def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=N
     rs, nr = _idx(rows, N)
     o = np.empty((nh, nr, d), np.float64)
     lse = np.empty((nh, nr), np.float64)
-    with _BlockMask(block_mask, H, N, block):
+    with _BlockMask(block_mask, H, N, block), _SeqLens(seqlens, B, N):
         rc = _load().orc_forward(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, f64,
                                  B, H, N, d, float(scale), int(bool(causal)), float(p_drop), int(seed),
                                  _p(hs, ctypes.c_int32), nh, _p(rs, ctypes.c_int32), nr,
@@ -187,7 +217,7 @@ def forward(q, k, v, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=N
 
 
 def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, rows=None,
-               block_mask=None, block=128):
+               block_mask=None, block=128, seqlens=None):
     """dQ_i and D_i for the selected query rows.
 
     Returns ``(dq, D, max_rel_dev)``; ``max_rel_dev`` is the largest relative
@@ -202,7 +232,7 @@ def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=Non
     dq = np.empty((nh, nr, d), np.float64)
     D = np.empty((nh, nr), np.float64)
     dev = ctypes.c_double(0.0)
-    with _BlockMask(block_mask, H, N, block):
+    with _BlockMask(block_mask, H, N, block), _SeqLens(seqlens, B, N):
         rc = _load().orc_backward_q(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
                                     db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
                                     float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,
@@ -214,7 +244,7 @@ def backward_q(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=Non
 
 
 def backward_kv(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=None, keys=None,
-                block_mask=None, block=128):
+                block_mask=None, block=128, seqlens=None):
     """dK_j and dV_j for the selected heads and key rows.
 
     Returns ``(dk, dv)`` of shape ``[nheads, nkeys, d]``.
@@ -226,7 +256,7 @@ def backward_kv(q, k, v, dout, scale, causal=False, p_drop=0.0, seed=0, heads=No
     ks, nk = _idx(keys, N)
     dk = np.empty((nh, nk, d), np.float64)
     dv = np.empty((nh, nk, d), np.float64)
-    with _BlockMask(block_mask, H, N, block):
+    with _BlockMask(block_mask, H, N, block), _SeqLens(seqlens, B, N):
         rc = _load().orc_backward_kv(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
                                      db.ctypes.data, f64, B, H, N, d, float(scale), int(bool(causal)),
                                      float(p_drop), int(seed), _p(hs, ctypes.c_int32), nh,

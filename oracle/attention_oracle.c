@@ -46,6 +46,14 @@
  *    optional mask over tile x tile blocks hides keys (s_ij = -inf); a row
  *    that sees no key at all gets P = 0, O = 0 and lse = -inf (the pages do
  *    not say; this is the limit of an empty softmax taken as zero weight).
+ *  - variable sequence lengths: "FlashAttention for Efficient Training",
+ *    section 5.2 (Handling Variable Sequence Lengths, Efficient Padding and
+ *    Masking: a score is -inf unless its key lies within the sequence,
+ *    j <= L_i with 1-based j).  An optional per-batch length L_b makes the
+ *    rows and keys at or beyond L_b of batch entry b padding: key j (0-based)
+ *    is visible to query i iff j < L_b, and a padding query row i >= L_b has
+ *    no keys at all (O = 0, lse = -inf, no gradient), so dK = dV = 0 for
+ *    padding keys.  Padding values never enter any result.
  * The pages print garbled dQ formulas; the dQ/dK expressions here are the
  * chain rule, pinned by finite differences in the tests.
  *
@@ -80,6 +88,8 @@ typedef struct {
      * queries i (hm = 0 if bmask_heads == 1, else the head h) */
     const uint8_t *bmask;
     int bmask_heads, bmask_tile;
+    /* optional lengths [B]: rows/keys >= seqlens[b] of batch entry b are padding */
+    const int32_t *seqlens;
 } problem_t;
 
 /* A row of one [B,H,N,d] input: base pointer plus its element type. */
@@ -180,14 +190,23 @@ static int block_masked(const problem_t *pb, int bh, int i, int j) {
     return pb->bmask[((size_t)hm * nt + (size_t)(i / pb->bmask_tile)) * nt + (size_t)(j / pb->bmask_tile)] == 0;
 }
 
+/* Number of real (non-padding) rows of the batch entry of head bh. */
+static int seq_len(const problem_t *pb, int bh) {
+    if (!pb->seqlens) return pb->N;
+    const int L = pb->seqlens[bh / pb->H];
+    return L < pb->N ? L : pb->N;
+}
+
 /* Scores s_ij for row i of head bh, then the row statistics m_i and l_i.
  * A row that sees no key (every key hidden by the block mask) has
  * m = -inf and l = 0; its probabilities are taken as 0. */
 static void row_scores(const problem_t *pb, int bh, int i, double *s, double *m_out, double *l_out) {
     row_t qi = row_ptr(pb, pb->q, bh, i);
+    const int L = seq_len(pb, bh);
     double m = -INFINITY;
     for (int j = 0; j < pb->N; ++j) {
-        if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {
+        /* a padding query sees no key; a padding key is seen by no query */
+        if (i >= L || j >= L || (pb->causal && j > i) || block_masked(pb, bh, i, j)) {
             s[j] = -INFINITY;
         } else {
             s[j] = pb->scale * dot_rows(qi, row_ptr(pb, pb->k, bh, j), pb->d);
@@ -278,6 +297,7 @@ static problem_t make_problem(const void *q, const void *k, const void *v, const
     pb.bmask = NULL;
     pb.bmask_heads = 1;
     pb.bmask_tile = 128;
+    pb.seqlens = NULL;
     return pb;
 }
 
@@ -293,10 +313,17 @@ void orc_set_block_mask(const uint8_t *mask, int heads, int tile) {
     tl_bmask_tile = tile > 0 ? tile : 128;
 }
 
+/* Per-batch lengths used by the next calls of this thread (NULL: every
+ * batch entry has all N rows).  lens is [B]. */
+static _Thread_local const int32_t *tl_seqlens = NULL;
+
+void orc_set_seqlens(const int32_t *lens) { tl_seqlens = lens; }
+
 static void apply_block_mask(problem_t *pb) {
     pb->bmask = tl_bmask;
     pb->bmask_heads = tl_bmask_heads;
     pb->bmask_tile = tl_bmask_tile;
+    pb->seqlens = tl_seqlens;
 }
 
 static int check_args(int B, int H, int N, int d, double p_drop) {
@@ -475,10 +502,12 @@ int orc_backward_kv(const void *q, const void *k, const void *v, const void *dou
             dkj[c] = 0.0;
             dvj[c] = 0.0;
         }
+        const int L = seq_len(&pb, bh);
+        if (j >= L) continue; /* a padding key: dK_j = dV_j = 0 */
         row_t kj = row_ptr(&pb, pb.k, bh, j);
         row_t vj = row_ptr(&pb, pb.v, bh, j);
         int i0 = causal ? j : 0;
-        for (int i = i0; i < N; ++i) {
+        for (int i = i0; i < L; ++i) {
             if (block_masked(&pb, bh, i, j)) continue;
             size_t su = (size_t)hi * nstat + (size_t)(i - first_row);
             row_t qi = row_ptr(&pb, pb.q, bh, i);

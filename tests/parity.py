@@ -1,0 +1,110 @@
+"""The parity bar shared by the GPU tests: the CUDA path against the fp64 oracle.
+
+Bounds (bf16 inputs and outputs, fp32 accumulation):
+  * O, dQ, dK, dV: max |err| <= 2e-2 and relative L2 error <= 5e-3;
+  * lse: max |err| <= 1e-3, and rows whose reference is -inf must be -inf;
+  * dropout keep masks: bit-exact (checked where they are compared).
+
+One recorded exception to the 2e-2 bound.  A bf16 output is the fp32 result
+rounded to the nearest bf16 value, and for |ref| >= 4 that rounding alone can
+take half an ulp, 2^-6 = 0.0156 in [4, 8) and twice that per binade above, so
+2e-2 leaves almost nothing for the arithmetic before the rounding.  Below
+|ref| = 4 the rounding takes at most 2^-7, and 2e-2 leaves 2e-2 - 2^-7 =
+0.0122 for that arithmetic.  The exception keeps that same allowance above 4:
+an element with |ref| >= 4 may exceed 2e-2 by up to
+    half_ulp(|ref|) + (2e-2 - 2^-7),
+and no more.  Every element that uses the exception is counted: ``check``
+records, per call, how many elements lie in (2e-2, that bound] and the worst
+one; the count may not exceed ``max(4, 1e-4 * elements)`` (so a systematic
+error cannot hide behind it); and the session prints every such record at
+the end (``tests/conftest.py``), and writes them as JSON lines to the file
+``FA_PARITY_REPORT`` names, if that variable is set.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+LSE_ABS = 1e-3
+# what 2e-2 leaves for the arithmetic before the final rounding below |ref| = 4
+PRE_ROUND = MAX_ABS - 2.0 ** -7
+EXC_FRACTION = 1e-4
+EXC_FLOOR = 4
+
+# one dict per check that used the exception (filled during the session)
+RECORDS: list = []
+_current_test = {"id": None}
+
+
+def set_current_test(nodeid: str) -> None:
+    _current_test["id"] = nodeid
+
+
+def half_ulp(x):
+    """Half a bf16 ulp at |x|: 2^(e - 8) for |x| in [2^e, 2^(e+1)) (8 significand bits)."""
+    _, e = np.frexp(np.abs(x))  # |x| = f * 2^e with f in [0.5, 1): binade [2^(e-1), 2^e)
+    return np.ldexp(1.0, e - 9)
+
+
+def element_bound(ref, scale: float = 1.0):
+    """The per-element absolute bound: 2e-2, or the recorded exception's
+    bound where |ref| >= 4.  ``scale`` > 1 widens both (only the random sweep
+    uses it, off the workloads' operating point)."""
+    b = np.where(np.abs(ref) >= 4.0, np.maximum(MAX_ABS, half_ulp(ref) + PRE_ROUND), MAX_ABS)
+    return b * scale
+
+
+def _record(rec: dict) -> None:
+    RECORDS.append(rec)
+    path = os.environ.get("FA_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def check(name, got, ref, exclude_rows=None, scale: float = 1.0):
+    """Max |err| and relative L2 of ``got`` (a torch tensor) against ``ref``.
+
+    ``exclude_rows`` (indices into axis -2) leaves rows out of the relative
+    metric only: rows whose exact value is identically zero, where a relative
+    error is undefined; they still meet the absolute bound.  An all-zero
+    reference is held to the absolute bound only, for the same reason.
+    """
+    g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    assert np.all(np.isfinite(g)), f"{name}: non-finite output"
+    err = np.abs(g - ref)
+    bound = element_bound(ref, scale)
+    worst = np.unravel_index(np.argmax(err / bound), err.shape) if err.size else ()
+    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert np.all(err <= bound), (f"{name}: abs err {err[worst]:.3e} at {worst} (|ref| {abs(ref[worst]):.3e}, "
+                                  f"bound {bound[worst]:.3e}), {int((err > bound).sum())} over, rel L2 {rel:.3e}")
+    over = err > MAX_ABS * scale
+    n_over = int(over.sum())
+    if n_over:
+        w = np.unravel_index(np.argmax(np.where(over, err, 0.0)), err.shape)
+        cap = max(EXC_FLOOR, int(EXC_FRACTION * err.size))
+        _record({"test": _current_test["id"], "tensor": name, "elements": int(err.size), "over_2e-2": n_over,
+                 "cap": cap, "worst_err": float(err[w]), "ref_at_worst": float(ref[w]),
+                 "bound_at_worst": float(bound[w]), "scale": scale})
+        assert n_over <= cap, f"{name}: {n_over} elements above {MAX_ABS * scale:g} (cap {cap})"
+    if exclude_rows:
+        keep = np.ones(ref.shape[-2], bool)
+        keep[list(exclude_rows)] = False
+        g, ref = g[..., keep, :], ref[..., keep, :]
+    if np.linalg.norm(ref) == 0.0:
+        return
+    rel = np.linalg.norm(g - ref) / np.linalg.norm(ref)
+    assert rel <= REL_L2, f"{name}: rel L2 err {rel:.3e}"
+
+
+def check_lse(got, ref):
+    g = got.detach().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    empty = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(g), empty), "lse: -inf rows differ"
+    if (~empty).any():
+        err = np.abs(g[~empty] - ref[~empty]).max()
+        assert err <= LSE_ABS, f"lse: max abs err {err:.3e}"

@@ -5,9 +5,10 @@ Each case draws B, H, N, d, the scale, causal, dropout, the tensor layout
 (plain, block-sparse with a random block mask, or split-KV forward) from one
 seeded generator, runs the CUDA path through the C ABI and compares every
 element with the oracle.  At the workloads' operating point (scale at most
-1/sqrt(d), dropout at most 0.1) the bar is the parity bar of every other test:
-max |err| <= 2e-2 (one bf16 ulp of |ref| where that is larger) and relative
-L2 <= 5e-3 for O, dQ, dK, dV, lse within 1e-3.  Draws beyond it (scale up to
+1/sqrt(d), dropout at most 0.1; three draws in four have such a scale) the bar
+is the parity bar of every other test (tests/parity.py): max |err| <= 2e-2 with
+the counted |ref| >= 4 rounding exception and relative L2 <= 5e-3 for O, dQ,
+dK, dV, lse within 1e-3.  Draws beyond it (scale up to
 1.5/sqrt(d), dropout 0.3) enlarge the bf16 rounding of dS and of the stored O
 that early causal rows concentrate on a few keys; there the absolute bound is
 doubled and the relative bound kept, which still fails any indexing, masking
@@ -20,34 +21,27 @@ import pytest
 import torch
 
 import oracle
+import parity
 from io_aware_exact_25_b200 import binding
 from io_aware_exact_25_b200.inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
 
-N_CASES = 24
+N_CASES = 32
+# absolute-bound factor for draws beyond the workloads' operating point
+WIDE = 2.0
+
+
+def _is_wide(c) -> bool:
+    """Beyond the operating point: scale above 1/sqrt(d) or dropout above 0.1."""
+    return c["scale"] * math.sqrt(c["d"]) > 1.0 or c["p"] > 0.1
 
 
 def _check(name, got, ref, wide=False):
-    g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
-    assert np.all(np.isfinite(g)), f"{name}: non-finite output"
-    err = np.abs(g - ref)
-    _, e = np.frexp(np.abs(ref))
-    bound = np.maximum(2e-2, np.ldexp(1.0, e - 8)) * (2.0 if wide else 1.0)
-    worst = np.unravel_index(np.argmax(err / bound), err.shape)
-    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-300)
-    assert np.all(err <= bound), (f"{name}: abs err {err[worst]:.3e} at {worst} (|ref| {abs(ref[worst]):.3e}), "
-                                  f"rel L2 {rel:.3e}")
-    if np.linalg.norm(ref) > 0:
-        assert rel <= 5e-3, f"{name}: rel L2 err {rel:.3e}"
+    parity.check(name, got, ref, scale=WIDE if wide else 1.0)
 
 
-def _check_lse(got, ref):
-    g = got.detach().cpu().numpy().astype(np.float64).reshape(ref.shape)
-    empty = np.isneginf(ref)
-    assert np.array_equal(np.isneginf(g), empty), "lse: -inf rows differ"
-    if (~empty).any():
-        assert np.abs(g[~empty] - ref[~empty]).max() <= 1e-3
+_check_lse = parity.check_lse
 
 
 def _draw(case):
@@ -58,7 +52,8 @@ def _draw(case):
     H = int(g.integers(1, 4))
     causal = bool(g.integers(0, 2))
     p = float(g.choice([0.0, 0.0, 0.1, 0.3]))
-    scale = float(g.uniform(0.5, 1.5)) / math.sqrt(d)
+    # three draws in four at the workloads' operating point (scale <= 1/sqrt(d))
+    scale = float(g.uniform(0.5, 1.0) if g.random() < 0.75 else g.uniform(1.0, 1.5)) / math.sqrt(d)
     layout = str(g.choice(["bhsd", "bshd"]))
     variant = str(g.choice(["plain", "plain", "blocksparse", "splitkv"]))
     nt = (N + 127) // 128
@@ -102,7 +97,7 @@ def test_random_case_matches_oracle(cuda_device, case):
     ro, rlse = oracle.forward(x["q"], x["k"], x["v"], c["scale"], **okw)
     rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], c["scale"], **okw)
     rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], c["scale"], **okw)
-    wide = c["scale"] * math.sqrt(d) > 1.0 or c["p"] > 0.1
+    wide = _is_wide(c)
     _check("O", o, ro, wide)
     _check_lse(lse, rlse)
     if c["p"] > 0 and c["causal"]:
@@ -135,5 +130,11 @@ def test_sweep_covers_every_option():
     assert {c["variant"] for c in cases} == {"plain", "blocksparse", "splitkv"}
     assert any(c["p"] > 0 for c in cases) and any(c["p"] == 0 for c in cases)
     assert any(c["N"] % 128 for c in cases)
-    narrow = [c for c in cases if c["scale"] * math.sqrt(c["d"]) <= 1.0 and c["p"] <= 0.1]
-    assert len(narrow) >= N_CASES // 3  # enough cases held to the full bar
+    wide = [k for k, c in enumerate(cases) if _is_wide(c)]
+    # the doubled bound never applies at the operating point (scale <= 1/sqrt(d),
+    # dropout <= 0.1), and at least a third of the sweep is held to the full bar
+    for k in wide:
+        c = cases[k]
+        assert c["scale"] * math.sqrt(c["d"]) > 1.0 or c["p"] > 0.1
+    assert N_CASES - len(wide) >= N_CASES // 3
+    print(f"random sweep: {len(wide)} of {N_CASES} cases use the doubled absolute bound: {wide}")

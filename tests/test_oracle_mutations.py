@@ -16,10 +16,13 @@ SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
 
 MUTANTS = {
     "drop_minus_D_in_dS": ("double ds = p * (dp - D);", "double ds = p * dp;"),
-    "causal_mask_transposed": ("if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
-                               "if ((pb->causal && j < i) || block_masked(pb, bh, i, j)) {"),
-    "causal_mask_off_by_one": ("if ((pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
-                               "if ((pb->causal && j >= i) || block_masked(pb, bh, i, j)) {"),
+    "causal_mask_transposed": ("(pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
+                               "(pb->causal && j < i) || block_masked(pb, bh, i, j)) {"),
+    "causal_mask_off_by_one": ("(pb->causal && j > i) || block_masked(pb, bh, i, j)) {",
+                               "(pb->causal && j >= i) || block_masked(pb, bh, i, j)) {"),
+    "length_mask_off_by_one": ("if (i >= L || j >= L ||", "if (i >= L || j > L ||"),
+    "padding_queries_see_keys": ("if (i >= L || j >= L ||", "if (j >= L ||"),
+    "padding_keys_get_gradients": ("if (j >= L) continue; /* a padding key", "if (j > L) continue; /* a padding key"),
     "lse_without_max": ("*lse = l > 0.0 ? m + log(l) : -INFINITY;", "*lse = l > 0.0 ? log(l) : -INFINITY;"),
     "dropout_scale_inverted": ("const double inv_keep = 1.0 / (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;",
                                "const double inv_keep = (1.0 - pb->p_drop);\n    for (int c = 0; c < pb->d; ++c) o[c] = 0.0;"),

@@ -453,3 +453,93 @@ def test_block_mask_shape_is_checked():
         oracle.forward(x["q"], x["k"], x["v"], 0.3, block_mask=np.ones((1, 4, 4), np.uint8), block=8)
     with pytest.raises(ValueError):
         oracle.forward(x["q"], x["k"], x["v"], 0.3, block_mask=np.ones((3, 5, 5), np.uint8), block=8)
+
+
+# ------------------------------------------------- variable sequence lengths
+#
+# "FlashAttention for Efficient Training", section 5.2 (Efficient Padding and
+# Masking): a score is -inf unless its key lies within the sequence.  With a
+# length L_b per batch entry, rows and keys at or beyond L_b are padding.
+
+def _varlen_all(x, sc, causal, lens, p=0.0, seed=0):
+    kw = dict(causal=causal, p_drop=p, seed=seed, seqlens=lens)
+    o, lse = oracle.forward(x["q"], x["k"], x["v"], sc, **kw)
+    dq, D, dev = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], sc, **kw)
+    dk, dv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], sc, **kw)
+    assert dev < 1e-12
+    return o, lse, dq, D, dk, dv
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_rows_equal_torch_on_each_unpadded_sequence(causal):
+    """Each batch entry's real rows equal torch fp64 SDPA + autograd run on
+    that sequence alone; padding rows are exactly O = 0, lse = -inf, dQ = 0
+    and padding keys exactly dK = dV = 0."""
+    B, H, N, d = 4, 2, 24, 8
+    lens = [24, 13, 1, 0]
+    x = make_inputs(B, H, N, d, seed=41)
+    sc = 0.35
+    o, lse, dq, D, dk, dv = _varlen_all(x, sc, causal, lens)
+    shape = (B, H, N, d)
+    o, dq, dk, dv = (t.reshape(shape) for t in (o, dq, dk, dv))
+    lse, D = lse.reshape(B, H, N), D.reshape(B, H, N)
+    for b, L in enumerate(lens):
+        pad = slice(L, N)
+        assert np.all(o[b, :, pad] == 0.0) and np.all(np.isneginf(lse[b, :, pad]))
+        assert np.all(dq[b, :, pad] == 0.0) and np.all(D[b, :, pad] == 0.0)
+        assert np.all(dk[b, :, pad] == 0.0) and np.all(dv[b, :, pad] == 0.0)
+        if L == 0:
+            continue
+        q, k, v = (_f64(x[n][b:b + 1, :, :L]).requires_grad_(True) for n in ("q", "k", "v"))
+        o_ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=sc)
+        o_ref.backward(_f64(x["do"][b:b + 1, :, :L]))
+        s = (q.detach() @ k.detach().transpose(-1, -2)) * sc
+        if causal:
+            s = s.masked_fill(~torch.ones(L, L, dtype=torch.bool).tril(), float("-inf"))
+        lse_ref = torch.logsumexp(s, dim=-1)[0].numpy()
+        assert np.max(np.abs(o[b, :, :L] - o_ref.detach()[0].numpy())) < 1e-12
+        assert np.max(np.abs(lse[b, :, :L] - lse_ref)) < 1e-12
+        for got, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+            assert np.max(np.abs(got[b, :, :L] - ref[0].numpy())) < 1e-11
+
+
+def test_varlen_padding_values_never_enter_a_result():
+    """Rewriting every padding row of Q, K, V and dO changes no bit of any
+    output."""
+    B, H, N, d = 3, 2, 20, 8
+    lens = [20, 7, 12]
+    x = make_inputs(B, H, N, d, seed=42)
+    y = {n: t.clone() for n, t in x.items()}
+    g = torch.Generator().manual_seed(43)
+    for b, L in enumerate(lens):
+        for n in y:
+            y[n][b, :, L:] = (torch.randn(H, N - L, d, generator=g) * 50).to(torch.bfloat16)
+    for causal in (False, True):
+        a = _varlen_all(x, 0.3, causal, lens, p=0.2, seed=9)
+        c = _varlen_all(y, 0.3, causal, lens, p=0.2, seed=9)
+        for u, w in zip(a, c):
+            assert np.array_equal(u, w)
+
+
+def test_varlen_with_equal_lengths_is_the_shorter_problem_with_dropout():
+    """All lengths L < N: the padded problem equals the unpadded N = L batch
+    bit for bit, dropout included (the mask is indexed by the batch entry and
+    the positions within the sequence)."""
+    B, H, N, d, L = 2, 2, 32, 8, 19
+    x = make_inputs(B, H, N, d, seed=44)
+    sub = {n: t[:, :, :L].contiguous() for n, t in x.items()}
+    for causal in (False, True):
+        a = _varlen_all(x, 0.4, causal, [L] * B, p=0.25, seed=11)
+        c = _varlen_all(sub, 0.4, causal, None, p=0.25, seed=11)
+        BH = B * H
+        for u, w in zip(a, c):
+            u = u.reshape(BH, N, -1) if u.ndim == 3 else u.reshape(BH, N, 1)
+            w = w.reshape(BH, L, -1) if w.ndim == 3 else w.reshape(BH, L, 1)
+            assert np.array_equal(u[:, :L], w)
+
+
+def test_varlen_lengths_are_checked():
+    x = make_inputs(2, 1, 8, 8, seed=45)
+    for bad in ([8], [9, 1], [-1, 3]):
+        with pytest.raises(ValueError):
+            oracle.forward(x["q"], x["k"], x["v"], 0.3, seqlens=bad)
