@@ -421,11 +421,23 @@ def run_ours(args, w):
     if binding.device_error(stream) != 0:
         raise RuntimeError("kernel reported a device error in the end-to-end run")
 
-    # max over ranks
-    from io_aware_exact_25_b200.replicas import max_over_ranks
-    times = max_over_ranks([elapsed_ms, e2e_ms] + per_stage_ms, device=dev)
-    elapsed_ms, e2e_ms = times[0], times[1]
-    per_stage_ms = times[2:]
+    # every replica checks its own outputs with identities that hold at any
+    # size (sum_j dK_j = 0 and, without dropout, sum_j dV_j = sum_i dO_i, in
+    # fp32 sums of the bf16 outputs; everything finite), then the job takes
+    # the slowest rank's times and the AND of the checks
+    ok = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
+              and torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all())
+    if mask is None:
+        sdk = dk.float().sum(dim=2)
+        ok = ok and bool((sdk.abs() <= 1e-2 * dk.float().abs().sum(dim=2) + 1e-2).all())
+        if w.p_drop == 0.0:
+            sdv, sdo = dv.float().sum(dim=2), do.float().sum(dim=2)
+            ok = ok and bool(((sdv - sdo).abs() <= 1e-2 * dv.float().abs().sum(dim=2) + 1e-2).all())
+    from io_aware_exact_25_b200.replicas import replica_summary
+    summ = replica_summary(elapsed_ms, e2e_ms, per_stage_ms, ok, device=dev)
+    elapsed_ms, e2e_ms, per_stage_ms = summ["elapsed_ms"], summ["e2e_ms"], summ["stage_ms"]
+    if not summ["all_ok"]:
+        raise RuntimeError("a replica's outputs failed their checks")
 
     if rank == 0:
         ff, fb = w.fwd_flops(), w.bwd_flops()
@@ -517,6 +529,8 @@ def run_ours(args, w):
                            "downloads on three streams over two device buffer sets"},
             "gpu_launches": args.steps * (len(stages) + (1 if splits > 1 else 0)),
             "splitkv": splits,
+            "replica_checks": {"ranks": ws, "all_ok": summ["all_ok"],
+                               "checks": "finite outputs; sum_j dK_j = 0; sum_j dV_j = sum_i dO_i without dropout"},
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

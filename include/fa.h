@@ -234,6 +234,91 @@ int fa_bwd_recompute_blocksparse(const void* q, const void* k, const void* v, co
                                  void* stream);
 
 /*
+ * Variable-length batches ("FlashAttention for Efficient Training" section
+ * 5.2, Handling Variable Sequence Lengths: a score is -inf unless its key lies
+ * within the sequence, j <= L_i, and no work is spent on padded tokens).
+ *  - Layout: the B sequences are stored token-major, the pages'
+ *    (batch, seq_len, num_heads, head_dim) layout with batch and sequence
+ *    folded into one token dimension of total_tokens rows: element (token t,
+ *    head h, c) of q, k, v, o (and dout, dq, dk, dv) is at
+ *    base[t * s.n + h * s.h + c], s = strides[i] (.b is ignored; .n and .h
+ *    times 2 bytes must be multiples of 16).  lse is fp32 [H, total_tokens].
+ *  - cu_seqlens: device int32 [B + 1], non-decreasing, 0 <= cu_seqlens[b] and
+ *    cu_seqlens[B] <= total_tokens; sequence b owns the slot of tokens
+ *    [cu_seqlens[b], cu_seqlens[b + 1]).  seqused: device int32 [B] or NULL;
+ *    if given, only the first seqused[b] tokens of the slot are the sequence
+ *    and the rest of the slot is padding (a padded [B, N, H, d] batch is
+ *    cu_seqlens = {0, N, 2N, ...} with seqused = the lengths); if NULL the
+ *    whole slot is the sequence.  max_seqlen (host) is at least the largest
+ *    slot size; it sizes the grid.
+ *  - Semantics per sequence b of length L_b: query i (position within the
+ *    sequence) sees key j iff j < L_b (and j <= i when causal); other
+ *    sequences are never seen.  Dropout uses hash32(seed, b, h, i, j) with
+ *    the positions within the sequence.  Padding rows (slot positions at or
+ *    beyond L_b) get o = 0 and lse = -inf, and dq = dk = dv = 0 in the
+ *    backward.  Every row of k and v inside a slot must hold finite values:
+ *    rows past L_b get zero weight, but the tensor cores multiply them by
+ *    that zero.
+ *  - Offsets are read on the device and not validated on the host; offsets
+ *    or lengths out of range are clamped into [0, total_tokens] and the slot
+ *    (so no access leaves the tensors) and reported as device error 3
+ *    (fa_get_device_error).
+ *  - Work, memory traffic and grid: CTAs of tiles past a sequence's length
+ *    return at once; the work is that of the B separate problems.
+ *  - The backward needs a workspace of fa_bwd_varlen_workspace_size bytes
+ *    and the forward's lse; its other arguments are those of fa_bwd_strided.
+ *  - Errors: as fa_fwd_strided / fa_bwd_strided; a null cu_seqlens is
+ *    FA_ERR_INVALID_ARG.  total_tokens = 0 is an empty problem.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                  const int32_t* cu_seqlens, const int32_t* seqused, int B, int H, int max_seqlen, int total_tokens,
+                  int d, float scale, int causal, float dropout_p, uint64_t seed, void* stream);
+size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen, int d);
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, const fa_strides* strides, const int32_t* cu_seqlens,
+                  const int32_t* seqused, int B, int H, int max_seqlen, int total_tokens, int d, float scale,
+                  int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/*
+ * Sequence parallelism over a split key range ("FlashAttention for Efficient
+ * Training" section 5.3, Sequence Parallelism for Long Contexts: each GPU
+ * holds a chunk of the sequence, and the output of a query chunk is formed
+ * from the softmax pieces of every key chunk, merged exactly by their
+ * logsumexp as in section 6.1's split-KV).  These entry points are the
+ * per-GPU pieces; io_aware_exact_25_b200/seqpar.py exchanges them over NCCL.
+ * A key window [kv_begin, kv_end) of the N keys has kv_begin a multiple of
+ * 128 and kv_end a multiple of 128 or N (else FA_ERR_INVALID_ARG); k, v, dk,
+ * dv of these calls are dense [B, H, kv_end - kv_begin, d] bf16 holding
+ * those key rows; q, dout are the full dense [B, H, N, d].
+ *
+ * fa_fwd_partial: for every query row, the softmax piece over the window's
+ *   keys: part_o fp32 [B, H, N, d] = O normalised over those keys and
+ *   part_lse fp32 [B, H, N] their logsumexp (-inf and O = 0 for a row that
+ *   sees none of them, e.g. causal rows before kv_begin).  Dropout uses the
+ *   global positions, so the pieces of all windows form one mask.
+ * fa_merge_partials: o bf16 [B, H, N, d] and lse [B, H, N] from num_parts
+ *   pieces stacked as part_o [num_parts][B, H, N, d], part_lse
+ *   [num_parts][B, H, N]: lse = ln sum_s e^lse_s, O = sum_s e^(lse_s - lse) O_s.
+ * fa_bwd_recompute_range: the recompute stage of fa_bwd for the window's
+ *   keys: writes dk, dv of those keys (complete) and adds their part of dQ
+ *   into the workspace's fp32 accumulator.  Run fa_bwd_prepare (on the full
+ *   o, dout, lse), this, then -- after summing the first
+ *   fa_bwd_dq_accumulator_bytes(B, H, N, d) bytes of the workspace (the
+ *   accumulator, fp32) over the windows that make up the sequence --
+ *   fa_bwd_finalize.  With one window covering every key this is fa_bwd.
+ */
+int fa_fwd_partial(const void* q, const void* k, const void* v, float* part_o, float* part_lse, int B, int H, int N,
+                   int d, float scale, int causal, float dropout_p, uint64_t seed, int kv_begin, int kv_end,
+                   void* stream);
+int fa_merge_partials(const float* part_o, const float* part_lse, int num_parts, void* o, float* lse, int B, int H,
+                      int N, int d, void* stream);
+size_t fa_bwd_dq_accumulator_bytes(int B, int H, int N, int d);
+int fa_bwd_recompute_range(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
+                           int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int kv_begin,
+                           int kv_end, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Debug export of the dropout mask: for each listed head bh = b*H + h
  * (heads[nheads]) and query row (rows[nrows]), writes the keep bit of every
  * key j < N to out[(hi * nrows + ri) * N + j] (1 = kept).  heads, rows and
@@ -265,7 +350,8 @@ int fa_last_cuda_error(void);
  * Synchronises `stream`, then reads and clears the calling device's error
  * word.  Returns 0 if no kernel reported an error since the last read, else
  * the kernel's code (1 = a bounded wait timed out, 2 = shared memory
- * misaligned); FA_ERR_CUDA if the synchronisation itself failed.
+ * misaligned, 3 = variable-length offsets or lengths out of range);
+ * FA_ERR_CUDA if the synchronisation itself failed.
  */
 int fa_get_device_error(void* stream);
 

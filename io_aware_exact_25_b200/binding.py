@@ -31,6 +31,8 @@ EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspa
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
            "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout",
+           "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
+           "fa_fwd_partial", "fa_merge_partials", "fa_bwd_dq_accumulator_bytes", "fa_bwd_recompute_range",
            "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -86,13 +88,24 @@ def load() -> ctypes.CDLL:
         lib.fa_bwd_finalize.argtypes = [vp, I, I, I, I, F, vp, SZ, vp]
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
         lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
+        lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64, vp]
+        lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64,
+                                      vp, SZ, vp]
+        lib.fa_bwd_varlen_workspace_size.argtypes = [I, I, I, I]
+        lib.fa_bwd_varlen_workspace_size.restype = SZ
+        lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp]
+        lib.fa_merge_partials.argtypes = [vp, vp, I, vp, vp, I, I, I, I, vp]
+        lib.fa_bwd_dq_accumulator_bytes.argtypes = [I, I, I, I]
+        lib.fa_bwd_dq_accumulator_bytes.restype = SZ
+        lib.fa_bwd_recompute_range.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp, SZ, vp]
         lib.fa_strerror.argtypes = [I]
         lib.fa_strerror.restype = ctypes.c_char_p
         lib.fa_get_device_error.argtypes = [vp]
         for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
                    lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
                    lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
-                   lib.fa_debug_fwd_timeout,
+                   lib.fa_debug_fwd_timeout, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
+                   lib.fa_merge_partials, lib.fa_bwd_recompute_range,
                    lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
             fn.restype = I
@@ -295,6 +308,170 @@ def bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, causal=False, scale=None, dro
                                int(seed), _stream(stream))
     _call(rc, "fa_bwd_noalloc")
     return dq, dk, dv
+
+
+def _check_varlen(ts, cu_seqlens, seqused):
+    """Token-major [T, H, d] bf16 CUDA tensors of one shape (d contiguous),
+    int32 CUDA offsets [B + 1] and optional int32 lengths [B]."""
+    shape = ts[0].shape
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (there is no CPU path)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v, o, dO must be bf16")
+        if t.dim() != 3 or t.shape != shape:
+            raise ValueError("variable-length tensors must be [total_tokens, H, d] of one shape")
+        if t.stride(-1) != 1:
+            raise ValueError("the head dimension must be contiguous")
+    for name, a, n in (("cu_seqlens", cu_seqlens, None), ("seqused", seqused, None)):
+        if a is None:
+            continue
+        if not a.is_cuda or a.dtype != torch.int32 or a.dim() != 1 or not a.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA vector")
+    B = cu_seqlens.numel() - 1
+    if B < 0:
+        raise ValueError("cu_seqlens needs B + 1 >= 1 entries")
+    if seqused is not None and seqused.numel() != B:
+        raise ValueError("seqused must have B entries")
+    return B
+
+
+def _tok_strides(*ts):
+    arr = (FaStrides * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = FaStrides(0, t.stride(1), t.stride(0))
+    return arr
+
+
+def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, seqused=None, causal=False, scale=None, dropout_p=0.0, seed=0,
+               o=None, lse=None, stream=None):
+    """O [T, H, d] and lse [H, T] of a variable-length batch via
+    ``fa_fwd_varlen``: sequence b is tokens ``cu_seqlens[b]`` to
+    ``cu_seqlens[b+1]`` of the token-major tensors (its first ``seqused[b]``
+    tokens if given); ``max_seqlen`` bounds the slot sizes."""
+    B = _check_varlen((q, k, v), cu_seqlens, seqused)
+    T, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    _check_varlen((q, o), cu_seqlens, seqused)
+    rc = load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _tok_strides(q, k, v, o),
+                              _ptr(cu_seqlens), _ptr(seqused), B, H, int(max_seqlen), T, d, float(scale),
+                              int(bool(causal)), float(dropout_p), int(seed), _stream(stream))
+    _call(rc, "fa_fwd_varlen")
+    return o, lse
+
+
+def bwd_varlen(q, k, v, o, dout, lse, cu_seqlens, max_seqlen, seqused=None, causal=False, scale=None,
+               dropout_p=0.0, seed=0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV [T, H, d] of a variable-length batch via ``fa_bwd_varlen``
+    (the forward's ``lse`` [H, T]); allocates the workspace with torch if not
+    given."""
+    B = _check_varlen((q, k, v, o, dout), cu_seqlens, seqused)
+    T, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_varlen((q, dq, dk, dv), cu_seqlens, seqused)
+    lib = load()
+    need = int(lib.fa_bwd_varlen_workspace_size(B, H, int(max_seqlen), d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib.fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _tok_strides(q, k, v, o, dout, dq, dk, dv), _ptr(cu_seqlens), _ptr(seqused), B, H,
+                           int(max_seqlen), T, d, float(scale), int(bool(causal)), float(dropout_p), int(seed),
+                           _ptr(workspace), int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _call(rc, "fa_bwd_varlen")
+    return dq, dk, dv
+
+
+def fwd_partial(q, k_win, v_win, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, part_o=None,
+                part_lse=None, stream=None):
+    """The softmax piece over the key window [kv_begin, kv_begin + len) of
+    every query row via ``fa_fwd_partial``: q dense [B,H,N,d]; k_win, v_win
+    dense [B,H,len,d] holding those key rows.  Returns (part_o fp32
+    [B,H,N,d], part_lse fp32 [B,H,N])."""
+    _check_inputs(q)
+    _check_dense(q, k_win, v_win)
+    B, H, N, d = q.shape
+    nk = k_win.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if part_o is None:
+        part_o = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if part_lse is None:
+        part_lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = load().fa_fwd_partial(_ptr(q), _ptr(k_win), _ptr(v_win), _ptr(part_o), _ptr(part_lse), B, H, N, d,
+                               float(scale), int(bool(causal)), float(dropout_p), int(seed), int(kv_begin),
+                               int(kv_begin + nk), _stream(stream))
+    _call(rc, "fa_fwd_partial")
+    return part_o, part_lse
+
+
+def merge_partials(part_o, part_lse, o=None, lse=None, stream=None):
+    """O (bf16) and lse from stacked softmax pieces part_o [S,B,H,N,d] and
+    part_lse [S,B,H,N] via ``fa_merge_partials``."""
+    S, B, H, N, d = part_o.shape
+    if part_o.dtype != torch.float32 or part_lse.dtype != torch.float32:
+        raise ValueError("partials are fp32")
+    if not (part_o.is_contiguous() and part_lse.is_contiguous()) or tuple(part_lse.shape) != (S, B, H, N):
+        raise ValueError("partials must be dense [S,B,H,N,d] and [S,B,H,N]")
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=part_o.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=part_o.device)
+    rc = load().fa_merge_partials(_ptr(part_o), _ptr(part_lse), S, _ptr(o), _ptr(lse), B, H, N, d, _stream(stream))
+    _call(rc, "fa_merge_partials")
+    return o, lse
+
+
+def dq_accumulator_bytes(B, H, N, d) -> int:
+    return int(load().fa_bwd_dq_accumulator_bytes(B, H, N, d))
+
+
+def bwd_prepare(o, dout, lse, workspace, stream=None):
+    """``fa_bwd_prepare`` on dense tensors (D, scaled lse, zeroed dQ accumulator)."""
+    _check_inputs(o, dout)
+    _check_dense(o, dout)
+    B, H, N, d = o.shape
+    _call(load().fa_bwd_prepare(_ptr(o), _ptr(dout), _ptr(lse), B, H, N, d, _ptr(workspace),
+                                int(workspace.numel() * workspace.element_size()), _stream(stream)), "fa_bwd_prepare")
+
+
+def bwd_recompute_range(q, k_win, v_win, dout, kv_begin, workspace, causal=False, scale=None, dropout_p=0.0, seed=0,
+                        dk=None, dv=None, stream=None):
+    """dK, dV of the key window and its dQ part (added into the workspace's
+    accumulator) via ``fa_bwd_recompute_range``."""
+    _check_inputs(q, dout)
+    _check_dense(q, dout, k_win, v_win)
+    B, H, N, d = q.shape
+    nk = k_win.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dk = torch.empty_like(k_win) if dk is None else dk
+    dv = torch.empty_like(v_win) if dv is None else dv
+    rc = load().fa_bwd_recompute_range(_ptr(q), _ptr(k_win), _ptr(v_win), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d,
+                                       float(scale), int(bool(causal)), float(dropout_p), int(seed), int(kv_begin),
+                                       int(kv_begin + nk), _ptr(workspace),
+                                       int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _call(rc, "fa_bwd_recompute_range")
+    return dk, dv
+
+
+def bwd_finalize(dq, workspace, scale, stream=None):
+    """``fa_bwd_finalize``: dq = scale * the workspace accumulator, bf16."""
+    _check_inputs(dq)
+    _check_dense(dq)
+    B, H, N, d = dq.shape
+    _call(load().fa_bwd_finalize(_ptr(dq), B, H, N, d, float(scale), _ptr(workspace),
+                                 int(workspace.numel() * workspace.element_size()), _stream(stream)),
+          "fa_bwd_finalize")
+    return dq
 
 
 def dropout_mask(B, H, N, dropout_p, seed, heads, rows, device="cuda", stream=None):

@@ -27,6 +27,10 @@
 //     computes the dQ_i partial dS K_j, which a warpgroup stages in shared
 //     memory and adds into the fp32 accumulator with bulk reductions;
 //  3. dQ = scale * accumulator, rounded to bf16.
+// Variable-length mode ("FlashAttention for Efficient Training" section 5.2):
+// sequences stored token-major at offsets cu_seqlens; a CTA's item is a key
+// tile of one sequence and head, it loops over that sequence's query tiles
+// only, and items past a sequence's real length do nothing.
 // Block-sparse mode ("FlashAttention for Efficient Training" section 3.2,
 // Block-Sparse Attention Support): the CTA of key tile j loops only over
 // the query tiles whose mask entry for j is nonzero (a bit set in shared
@@ -75,11 +79,23 @@ struct BwdArgs {
   float* dq_acc;  // [BH, N, D] fp32 scratch
   float* lse2;    // [BH, Npad] scratch: lse * log2(e), +inf on padded rows
   float* drow;    // [BH, Npad] scratch: D_i, 0 on padded rows
+  int* sched;     // scratch: the persistent grid's item counter and done count
+                  // (zeroed by the row pass; the kernel leaves them zero)
   int* err;
   // block-sparse (SPARSE kernels only): bmask[hm][qt][kt] != 0 lets query
   // tile qt see key tile kt; hm = 0 when bmask_heads == 1, else the head
   const uint8_t* bmask;
   int bmask_heads;
+  // variable-length (VARLEN kernels; the row pass and dQ conversion test
+  // cu_seqlens at run time): token offsets [B+1], optional used lengths [B],
+  // token count T; N holds the largest slot size; lse is [H, T]
+  const int* cu_seqlens;
+  const int* seqused;
+  int total_tokens;
+  // key window: only key tiles [kv_lo, kv_hi) are processed (a rank's key
+  // chunk); the K, V, dK, dV tensors hold key rows from kv_row_off on, and
+  // the dQ accumulator receives the partial over those keys only
+  int kv_lo, kv_hi, kv_row_off;
 };
 
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -88,13 +104,14 @@ __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a -
 // tile by tile -- for each head, 128-row query tile and 16-column piece, one
 // contiguous 8 KB block of 128 rows x 16 columns whose 16-byte chunks are
 // permuted by the 64-byte swizzle (chunk k of row r at k ^ ((r >> 1) & 3)) --
-// then the scaled lse and D row vectors.
+// then the scaled lse and D row vectors, then the item counter.
 inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   const size_t npad = round_up((size_t)N, 128);
-  return round_up((size_t)BH * npad * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256);
+  return round_up((size_t)BH * npad * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256) + 256;
 }
 
-inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, float** lse2, float** drow) {
+inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, float** lse2, float** drow,
+                                int** sched) {
   const size_t npad = round_up((size_t)N, 128);
   char* p = static_cast<char*>(ws);
   *dq_acc = reinterpret_cast<float*>(p);
@@ -102,6 +119,8 @@ inline void bwd_workspace_split(void* ws, int BH, int N, int d, float** dq_acc, 
   *lse2 = reinterpret_cast<float*>(p);
   p += round_up((size_t)BH * npad * 4, 256);
   *drow = reinterpret_cast<float*>(p);
+  p += round_up((size_t)BH * npad * 4, 256);
+  *sched = reinterpret_cast<int*>(p);
 }
 
 // ------------------------------------------------------------ row pass
@@ -129,11 +148,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
       if (r < rows) {
         const int bh = (int)(r / npad);
         const int i = (int)(r - (long long)bh * npad);
-        if (i < a.N) {
-          const int b_ = bh / a.H, h_ = bh - b_ * a.H;
-          ov[u] = *reinterpret_cast<const uint4*>(a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + 8 * part);
-          dv[u] = *reinterpret_cast<const uint4*>(a.dout + b_ * a.do_sb + h_ * a.do_sh + (long long)i * a.do_sn +
-                                                  8 * part);
+        const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+        int len = a.N, row0 = 0;
+        if (a.cu_seqlens) {
+          const SeqSpan sp = varlen_span(a.cu_seqlens, a.seqused, b_, a.total_tokens, a.N, nullptr, false);
+          len = sp.len;
+          row0 = sp.row0;
+        }
+        if (i < len) {
+          const long long row = row0 + i;
+          ov[u] = *reinterpret_cast<const uint4*>(a.o + b_ * a.o_sb + h_ * a.o_sh + row * a.o_sn + 8 * part);
+          dv[u] = *reinterpret_cast<const uint4*>(a.dout + b_ * a.do_sb + h_ * a.do_sh + row * a.do_sn + 8 * part);
         }
       }
     }
@@ -150,10 +175,22 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
       if (part == 0 && r < rows) {
         const int bh = (int)(r / npad);
         const int i = (int)(r - (long long)bh * npad);
-        a.drow[r] = i < a.N ? acc : 0.f;
-        a.lse2[r] = i < a.N ? a.lse[(size_t)bh * a.N + i] * 1.4426950408889634f : INFINITY;
+        int len = a.N;
+        long long lse_at = (long long)bh * a.N + i;
+        if (a.cu_seqlens) {
+          const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+          const SeqSpan sp = varlen_span(a.cu_seqlens, a.seqused, b_, a.total_tokens, a.N, nullptr, false);
+          len = sp.len;
+          lse_at = (long long)h_ * a.total_tokens + sp.row0 + i;
+        }
+        a.drow[r] = i < len ? acc : 0.f;
+        a.lse2[r] = i < len ? a.lse[lse_at] * 1.4426950408889634f : INFINITY;
       }
     }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.sched[0] = 0;  // items drawn
+    a.sched[1] = 0;  // CTAs done drawing
   }
   const long long n4 = (long long)BH * npad * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(a.dq_acc);
@@ -166,7 +203,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                        int BH, int H, int N, long long sb, long long sh, long long sn,
-                                                       float scale) {
+                                                       float scale, const int* cu_seqlens, const int* seqused,
+                                                       int total_tokens) {
   const int npad = (N + 127) & ~127;
   const long long n8 = (long long)BH * N * (D / 8);
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n8;
@@ -179,6 +217,13 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     const int piece = c8 >> 1;            // 16-column piece
     const int k0 = (c8 & 1) * 2;          // first of the two 4-column chunks
     const int sw = (r >> 1) & 3;
+    const int b_ = bh / H, h_ = bh - b_ * H;
+    long long row = i;
+    if (cu_seqlens) {
+      const SeqSpan sp = varlen_span(cu_seqlens, seqused, b_, total_tokens, N, nullptr, false);
+      if (i >= sp.len) continue;  // padding rows are filled separately
+      row = sp.row0 + i;
+    }
     const float* blk = acc + (((size_t)bh * (npad >> 7) + tile) * (D / 16) + piece) * 2048 + r * 16;
     const float4 x = *reinterpret_cast<const float4*>(blk + ((k0 ^ sw) << 2));
     const float4 y = *reinterpret_cast<const float4*>(blk + (((k0 + 1) ^ sw) << 2));
@@ -187,8 +232,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     w.y = pack_bf16x2(x.z * scale, x.w * scale);
     w.z = pack_bf16x2(y.x * scale, y.y * scale);
     w.w = pack_bf16x2(y.z * scale, y.w * scale);
-    const int b_ = bh / H, h_ = bh - b_ * H;
-    *reinterpret_cast<uint4*>(dq + b_ * sb + h_ * sh + (long long)i * sn + 8 * c8) = w;
+    *reinterpret_cast<uint4*>(dq + b_ * sb + h_ * sh + row * sn + 8 * c8) = w;
   }
 }
 
@@ -217,9 +261,12 @@ struct BwdLayout {
   static constexpr uint32_t kOffDQ = (kOffRow + kRowStages * kRowStage + 1023u) & ~1023u;
   static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
-  // row_empty[2], s, dp, p, ds, kv_free, dk, dq, dq_free, drain, acc_free
-  static constexpr int kNumBars = 1 + 12 + 10;
-  static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
+  // row_empty[2], s, dp, p, ds, kv_free, dk, dq, dq_free, drain, acc_free,
+  // item_full[2], item_empty[2]
+  static constexpr int kNumBars = 1 + 12 + 10 + 4;
+  // after the barriers: TMEM address, abort flag, dQ-warpgroup flag, two item
+  // slots, the dQ warpgroup's item
+  static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 32;
   // block-sparse: the query-tile bit set and its count after the barriers
   static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
   static constexpr uint32_t kSmemSparse = kOffBits + kSparseWords * 4u + 16u;
@@ -240,7 +287,7 @@ __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk
 // exponential on the FMA pipe (polynomial), the rest on MUFU.
 constexpr int kBwdPolyPairsOf8 = 0;
 
-template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE, bool VARLEN>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -269,33 +316,69 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* bar_dq_free = bars + 20;
   uint64_t* bar_drain = bars + 21;
   uint64_t* bar_acc_free = bars + 22;  // dV/dK accumulators read out by the epilogue
+  uint64_t* bar_item_full = bars + 23;   // [2] the producer published the next item
+  uint64_t* bar_item_empty = bars + 25;  // [2] every role has read it (10 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);  // [0] abort, [1] dQ warpgroup flag
+  int* item_slot = abort_flag + 2;                           // [2] published item indices
+  int* dq_item = abort_flag + 4;                             // the dQ warpgroup's current item
   const uint32_t sbase = smem_u32(smem);
 
   const int BH = a.B * a.H;
   const int nT = (a.N + 127) >> 7;
   const int npad = nT * 128;
-  // Work items (key tile, head) in longest-processing-time order: key tiles
-  // ascending (the most query tiles first when causal), heads interleaved, so
-  // the CTAs working at one time sweep the query tiles of their heads in near
-  // lockstep and the Q/dO tiles and accumulator rows they share stay in L2.
-  // The grid is persistent: each CTA takes one item per round (see
-  // item_index); the next item's first products overlap the last item's dQ
-  // reductions and dK/dV write-out.  (Block-sparse kernels run one item per
-  // CTA.)
-  const int n_items = BH * nT;
+  // Work items are (key tile, head) pairs.  Their order groups the heads, hg
+  // at a time, and within a group
+  // puts the key tiles in ascending order with the group's heads interleaved:
+  // longest first when causal.  CTAs take items in this order -- the
+  // persistent grid from a counter in the workspace, one-item-per-CTA grids
+  // by block index, which the hardware dispatches in order -- so the items
+  // running at any time belong to a few heads, whose Q, dO and fp32 dQ
+  // accumulator stay in L2, and the short items of a group fill the time its
+  // long items leave.  In the persistent grid the next item's first products
+  // overlap the last item's dQ reductions and dK/dV write-out.
+  const int kt_hi = min(a.kv_hi, nT), kt_lo = min(a.kv_lo, kt_hi);
+  const int nTr = kt_hi - kt_lo;  // key tiles in the window
+  const int n_items = BH * nTr;
+  // Group size: a group holds about one CTA's share of the running items'
+  // work per SM (hg >= SMs / average item length, in query tiles); the heads
+  // left over join the last group, so the last group -- whose long items
+  // start last -- always holds at least that much work and the tail stays
+  // short.
+  uint32_t n_sm;
+  asm("mov.u32 %0, %%nsmid;" : "=r"(n_sm));
+  const int avg_len = max(1, CAUSAL ? nT - (kt_lo + kt_hi - 1) / 2 : nT);
+  const int hg = min(BH, max(1, ((int)n_sm + avg_len - 1) / avg_len));
+  const int n_groups = max(1, BH / hg);
+  // An item's sequence: real rows [0, len) at tokens row0.. of the tensors,
+  // batch coordinate wc of the tensor maps (variable-length: 0).
   struct Item {
-    int jt, bh, bb, hh, i_begin, n_steps;
+    int jt, bh, bb, hh, i_begin, n_steps, row0, len, wc;
   };
   auto item_of = [&](int w) {
+    const int grp = min(w / (hg * nTr), n_groups - 1);
+    const int h0 = grp * hg;
+    const int nh = grp == n_groups - 1 ? BH - h0 : hg;  // the last group takes the rest
+    const int r = w - h0 * nTr;
+    const int jl = r / nh;  // key tile within the window
     Item t;
-    t.jt = w / BH;
-    t.bh = w - t.jt * BH;
+    t.jt = kt_lo + jl;
+    t.bh = h0 + (r - jl * nh);
     t.bb = t.bh / a.H;
     t.hh = t.bh - t.bb * a.H;
     t.i_begin = CAUSAL ? t.jt : 0;
     t.n_steps = nT - t.i_begin;
+    t.row0 = 0;
+    t.len = a.N;
+    t.wc = t.bb;
+    if (VARLEN) {
+      const SeqSpan sp = varlen_span(a.cu_seqlens, a.seqused, t.bb, a.total_tokens, a.N, a.err, t.jt == 0);
+      t.row0 = sp.row0;
+      t.len = sp.len;
+      t.wc = 0;
+      const int nTb = (sp.len + 127) >> 7;
+      t.n_steps = t.jt < nTb ? nTb - t.i_begin : 0;
+    }
     return t;
   };
   uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // SPARSE: query tiles that see jt
@@ -322,6 +405,10 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_dq, 1);
     mbar_init(bar_dq_free, 128);
     mbar_init(bar_drain, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_item_full[s], 1);
+      mbar_init(&bar_item_empty[s], 10);  // MMA thread, dQ leader, 8 P/dS warps
+    }
     const bool misaligned = (sbase & 1023u) != 0u;
     *abort_flag = misaligned ? 1 : 0;
     if (misaligned && a.err) atomicCAS(a.err, kDevOk, kDevMisaligned);
@@ -345,17 +432,19 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, a.err};
   const bool run = *abort_flag == 0;
-  // Item of round r for this CTA: rounds alternate direction across the grid
-  // ("snake" order), so with items sorted by decreasing length every CTA gets
-  // nearly the same total work.
-  // Dropout and block-sparse kernels run one item per CTA (see the launch);
-  // for them the loops below make a single pass that the compiler folds.
-  constexpr bool PERSIST = !SPARSE && !DROPOUT;
-  const int n_rounds = PERSIST ? (n_items + (int)gridDim.x - 1) / (int)gridDim.x : 1;
-  auto item_index = [&](int r) {
-    if (!PERSIST) return (int)blockIdx.x;
-    const int G = (int)gridDim.x, c = (int)blockIdx.x;
-    return r * G + ((r & 1) ? (G - 1 - c) : c);
+  // Dropout, variable-length and block-sparse kernels run one item per CTA
+  // (see the launch); for them the loops below make a single pass.
+  constexpr bool PERSIST = !SPARSE && !DROPOUT && !VARLEN;
+  // Item r of this CTA for a consuming role: the persistent grid reads the
+  // slot the producer published (the caller then arrives on
+  // bar_item_empty[r & 1]); n_items ends the loop.
+  auto peek_item = [&](int r, bool& ok_) -> int {
+    if (!PERSIST) return r == 0 ? (int)blockIdx.x : n_items;
+    if (!mbar_wait(&bar_item_full[r & 1], (uint32_t)(r >> 1) & 1u, ab)) {
+      ok_ = false;
+      return n_items;
+    }
+    return *reinterpret_cast<volatile int*>(&item_slot[r & 1]);
   };
   // the items of this CTA, with the block-sparse step count
   auto item_at = [&](int w) {
@@ -380,17 +469,42 @@ __global__ void __launch_bounds__(448, 1)
     int q_issued = 0, do_issued = 0, kv_issued = 0;
     int g = 0;
     bool ok = true;
-    for (int r = 0; r < n_rounds && ok; ++r) {
-      const int w = item_index(r);
-      if (w >= n_items) continue;
+    for (int r = 0; ok; ++r) {
+      int w = 0;
+      if (PERSIST) {
+        // take the next item from the counter and publish it to the other roles
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_item_empty[r & 1], ((uint32_t)(r >> 1) & 1u) ^ 1u, ab))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          w = min(atomicAdd(a.sched, 1), n_items);
+          item_slot[r & 1] = w;
+          mbar_arrive(&bar_item_full[r & 1]);
+        }
+        w = __shfl_sync(0xffffffffu, w, 0);
+      } else {
+        w = r == 0 ? (int)blockIdx.x : n_items;
+      }
+      if (w >= n_items) {
+        // The last CTA to draw the end of the items resets the counter (and
+        // this count), so the next launch on the workspace starts from zero
+        // without a row pass: every CTA has drawn its last value by then.
+        if (PERSIST && lane == 0 && atomicAdd(a.sched + 1, 1) == (int)gridDim.x - 1) {
+          atomicExch(a.sched, 0);
+          atomicExch(a.sched + 1, 0);
+        }
+        break;
+      }
       const Item t = item_at(w);
       if (t.n_steps == 0) continue;  // (a key tile no query tile sees loads nothing)
       auto load_kv = [&]() {
         if (lane == 0) {
           mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
           for (int h = 0; h < D / 64; ++h) {
-            tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
-            tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, t.jt * 128, t.hh, t.bb, bar_kv, pol_keep);
+            const int krow = t.row0 + t.jt * 128 - a.kv_row_off;
+            tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, krow, t.hh, t.wc, bar_kv, pol_keep);
+            tma_load_4d(smem + L::kOffV + h * L::kHalf, &tm_v, 64 * h, krow, t.hh, t.wc, bar_kv, pol_keep);
           }
         }
         ++kv_issued;
@@ -409,8 +523,8 @@ __global__ void __launch_bounds__(448, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, i * 128, t.hh, t.bb,
-                        &bar_q_full[qs], pol_keep);
+            tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, t.row0 + i * 128, t.hh,
+                        t.wc, &bar_q_full[qs], pol_keep);
         }
         ++q_issued;
         const int ds_ = gs % L::kDoStages;
@@ -421,8 +535,8 @@ __global__ void __launch_bounds__(448, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&bar_do_full[ds_], L::kTile);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, i * 128, t.hh, t.bb,
-                        &bar_do_full[ds_], pol_keep);
+            tma_load_4d(smem + L::kOffDO + ds_ * L::kTile + h * L::kHalf, &tm_do, 64 * h, t.row0 + i * 128, t.hh,
+                        t.wc, &bar_do_full[ds_], pol_keep);
         }
         ++do_issued;
         // row statistics of query tile i
@@ -486,9 +600,10 @@ __global__ void __launch_bounds__(448, 1)
       // starts while dK(i) runs.  Across items the same order holds: the next
       // item's S(0) is queued behind the last dK, its first dV and dK (which
       // overwrite the accumulators) wait for the epilogue to have read them.
-      for (int r = 0; r < n_rounds && ok; ++r) {
-      const int w = item_index(r);
-      if (w >= n_items) continue;
+      for (int r = 0; ok; ++r) {
+        const int w = peek_item(r, ok);
+        if (PERSIST && ok) mbar_arrive(&bar_item_empty[r & 1]);
+        if (w >= n_items) break;
         const Item t = item_at(w);
         if (t.n_steps == 0) continue;
         ok = mbar_wait(bar_kv, kv_used & 1, ab) && mbar_wait(&bar_q_full[g & 1], (g >> 1) & 1, ab);
@@ -617,9 +732,22 @@ __global__ void __launch_bounds__(448, 1)
     };
     int g = 0;
     bool ok = true;
-    for (int r = 0; r < n_rounds && ok; ++r) {
-      const int w = item_index(r);
-      if (w >= n_items) continue;
+    for (int r = 0; ok; ++r) {
+      // the leader reads the item and shares it through shared memory
+      if (leader) {
+        bool ok_ = true;
+        const int w_ = peek_item(r, ok_);
+        if (PERSIST && ok_) mbar_arrive(&bar_item_empty[r & 1]);
+        *dq_item = ok_ ? w_ : -1;
+      }
+      named_bar_sync(1, 128);
+      const int w = *reinterpret_cast<volatile int*>(dq_item);
+      named_bar_sync(1, 128);  // everyone has read it before the leader may overwrite it
+      if (w < 0) {
+        ok = false;
+        break;
+      }
+      if (w >= n_items) break;
     const Item t = item_at(w);
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
@@ -698,13 +826,15 @@ __global__ void __launch_bounds__(448, 1)
     const float sl2 = a.scale_log2;
     bool ok = true;
     int g = 0;
-    for (int r = 0; r < n_rounds && ok; ++r) {
-      const int w = item_index(r);
-      if (w >= n_items) continue;
+    for (int r = 0; ok; ++r) {
+      const int w = peek_item(r, ok);
+      __syncwarp();
+      if (PERSIST && ok && lane == 0) mbar_arrive(&bar_item_empty[r & 1]);
+      if (!ok || w >= n_items) break;
     const Item t = item_at(w);
     const int jt = t.jt, bb = t.bb, hh = t.hh;
     const int key = jt * 128 + jr;
-    const bool key_ok = key < a.N;
+    const bool key_ok = key < t.len;
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
       const int i = SPARSE ? walk.next() : t.i_begin + it;
@@ -857,8 +987,9 @@ __global__ void __launch_bounds__(448, 1)
     if (!ok) break;
     if (SPARSE && t.n_steps == 0) {
       // no query tile sees this key tile
-      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + (long long)key * a.dv_sn
-                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + (long long)key * a.dk_sn;
+      const long long zrow = t.row0 + key - a.kv_row_off;
+      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + zrow * a.dv_sn
+                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + zrow * a.dk_sn;
       if (key_ok) {
 #pragma unroll
         for (int c = 0; c < D; c += 8) st_global_v4(dst + c, 0u, 0u, 0u, 0u);
@@ -871,8 +1002,9 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_after();
       const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
       const float mul = wg == 0 ? 1.f : a.scale;
-      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + (long long)(key_ok ? key : 0) * a.dv_sn
-                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + (long long)(key_ok ? key : 0) * a.dk_sn;
+      const long long krow = t.row0 + (key_ok ? key : jt * 128) - a.kv_row_off;
+      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + krow * a.dv_sn
+                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + krow * a.dk_sn;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t v[32];
@@ -902,20 +1034,24 @@ __global__ void __launch_bounds__(448, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE>
+template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE, bool VARLEN>
 cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const BwdArgs& a, cudaStream_t st) {
   using L = BwdLayout<D, DROPOUT>;
-  auto kern = bwd_kernel<D, CAUSAL, DROPOUT, SPARSE>;
+  auto kern = bwd_kernel<D, CAUSAL, DROPOUT, SPARSE, VARLEN>;
   const int smem = (int)(SPARSE ? L::kSmemSparse : L::kSmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  // One CTA per SM looping over the work items.  Block-sparse and dropout
-  // kernels run one CTA per item: block-sparse items differ in length in ways
-  // only the mask knows, and with dropout (one row-statistics stage at
-  // d = 128) the persistent grid measured 10% slower on N = 65536.
-  long long grid = (long long)a.B * a.H * ((a.N + 127) / 128);
-  if (!SPARSE && !DROPOUT) {
+  // One CTA per SM looping over the work items.  Block-sparse, variable-length
+  // and dropout kernels run one CTA per item: block-sparse and variable-length
+  // items differ in length in ways only device data knows, and with dropout
+  // (one row-statistics stage at d = 128) the persistent grid measured 10%
+  // slower on N = 65536.
+  const int nT = (a.N + 127) / 128;
+  const int kt_hi = a.kv_hi < nT ? a.kv_hi : nT, kt_lo = a.kv_lo < kt_hi ? a.kv_lo : kt_hi;
+  long long grid = (long long)a.B * a.H * (kt_hi - kt_lo);
+  if (grid == 0) return cudaSuccess;
+  if (!SPARSE && !DROPOUT && !VARLEN) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0 && grid > sms)
@@ -935,34 +1071,37 @@ inline cudaError_t launch_bwd_prepare(const BwdArgs& a, int d, cudaStream_t st) 
   return cudaGetLastError();
 }
 
-template <int D, bool SPARSE>
+template <int D, bool SPARSE, bool VARLEN>
 cudaError_t launch_bwd_recompute_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                    const CUtensorMap& mdo, const BwdArgs& a, bool causal,
                                    bool dropout, cudaStream_t st) {
   if (causal)
-    return dropout ? launch_bwd_main<D, true, true, SPARSE>(mq, mk, mv, mdo, a, st)
-                   : launch_bwd_main<D, true, false, SPARSE>(mq, mk, mv, mdo, a, st);
-  return dropout ? launch_bwd_main<D, false, true, SPARSE>(mq, mk, mv, mdo, a, st)
-                 : launch_bwd_main<D, false, false, SPARSE>(mq, mk, mv, mdo, a, st);
+    return dropout ? launch_bwd_main<D, true, true, SPARSE, VARLEN>(mq, mk, mv, mdo, a, st)
+                   : launch_bwd_main<D, true, false, SPARSE, VARLEN>(mq, mk, mv, mdo, a, st);
+  return dropout ? launch_bwd_main<D, false, true, SPARSE, VARLEN>(mq, mk, mv, mdo, a, st)
+                 : launch_bwd_main<D, false, false, SPARSE, VARLEN>(mq, mk, mv, mdo, a, st);
 }
 
 inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                         const CUtensorMap& mdo, const BwdArgs& a, int d,
                                         bool causal, bool dropout, cudaStream_t st) {
   if (a.bmask)
-    return d == 64 ? launch_bwd_recompute_d<64, true>(mq, mk, mv, mdo, a, causal, dropout, st)
-                   : launch_bwd_recompute_d<128, true>(mq, mk, mv, mdo, a, causal, dropout, st);
-  return d == 64 ? launch_bwd_recompute_d<64, false>(mq, mk, mv, mdo, a, causal, dropout, st)
-                 : launch_bwd_recompute_d<128, false>(mq, mk, mv, mdo, a, causal, dropout, st);
+    return d == 64 ? launch_bwd_recompute_d<64, true, false>(mq, mk, mv, mdo, a, causal, dropout, st)
+                   : launch_bwd_recompute_d<128, true, false>(mq, mk, mv, mdo, a, causal, dropout, st);
+  if (a.cu_seqlens)
+    return d == 64 ? launch_bwd_recompute_d<64, false, true>(mq, mk, mv, mdo, a, causal, dropout, st)
+                   : launch_bwd_recompute_d<128, false, true>(mq, mk, mv, mdo, a, causal, dropout, st);
+  return d == 64 ? launch_bwd_recompute_d<64, false, false>(mq, mk, mv, mdo, a, causal, dropout, st)
+                 : launch_bwd_recompute_d<128, false, false>(mq, mk, mv, mdo, a, causal, dropout, st);
 }
 
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
   if (d == 64)
     bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                 a.scale);
+                                                 a.scale, a.cu_seqlens, a.seqused, a.total_tokens);
   else
     bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                  a.scale);
+                                                  a.scale, a.cu_seqlens, a.seqused, a.total_tokens);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,9 @@ __device__ int g_device_error;  // kernels record kDevTimeout / kDevMisaligned h
 
 thread_local int t_last_cuda_error = 0;
 
+// Key-window upper bound meaning "every key tile".
+constexpr int kAllTiles = 1 << 30;
+
 int cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return FA_ERR_CUDA;
@@ -120,7 +123,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   kern<<<(unsigned)grid, L::kThreads, smem, st>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
-  if (SPLIT) {
+  if (SPLIT && !a.partial_only) {
     fa::splitkv_combine_kernel<D><<<148 * 8, 256, 0, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
@@ -165,11 +168,75 @@ __global__ void dropout_mask_kernel(int H, int N, uint32_t threshold, uint64_t s
   }
 }
 
+// Variable-length batches with padded slots (seqused given): the slot rows
+// [L_b, slot) of sequence b are padding.  Writes zeros into those rows of up
+// to three bf16 tensors (null entries are skipped) and -inf into lse rows of
+// a forward (lse may be null).  One thread per (sequence, slot row, head).
+__global__ void varlen_pad_kernel(int B, int H, int max_slot, int total, const int* cu, const int* used, int d,
+                                  __nv_bfloat16* t0, fa_strides s0, __nv_bfloat16* t1, fa_strides s1,
+                                  __nv_bfloat16* t2, fa_strides s2, float* lse) {
+  const long long n = (long long)B * max_slot * H;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n; u += (long long)gridDim.x * blockDim.x) {
+    const int h = (int)(u % H);
+    const long long br = u / H;
+    const int r = (int)(br % max_slot);
+    const int b = (int)(br / max_slot);
+    const fa::SeqSpan sp = fa::varlen_span(cu, used, b, total, max_slot, nullptr, false);
+    if (r < sp.len || r >= sp.slot) continue;
+    const long long row = sp.row0 + r;
+    __nv_bfloat16* ts[3] = {t0, t1, t2};
+    const fa_strides ss[3] = {s0, s1, s2};
+    for (int k = 0; k < 3; ++k) {
+      if (!ts[k]) continue;
+      __nv_bfloat16* p = ts[k] + h * ss[k].h + row * ss[k].n;
+      for (int c = 0; c < d; c += 8) *reinterpret_cast<uint4*>(p + c) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (lse) lse[(long long)h * total + row] = -INFINITY;
+  }
+}
+
+int launch_varlen_pad(int B, int H, int max_slot, int total, const int* cu, const int* used, int d,
+                      __nv_bfloat16* t0, fa_strides s0, __nv_bfloat16* t1, fa_strides s1, __nv_bfloat16* t2,
+                      fa_strides s2, float* lse, cudaStream_t st) {
+  varlen_pad_kernel<<<148 * 4, 256, 0, st>>>(B, H, max_slot, total, cu, used, d, t0, s0, t1, s1, t2, s2, lse);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+// Token-major strides {.n = token, .h = head} of a variable-length tensor as
+// the 4-D {d, T, H, 1} tensor maps and the kernels take them (.b unused).
+fa_strides varlen_strides(const fa_strides& s, int total) {
+  fa_strides r;
+  r.n = s.n;
+  r.h = s.h;
+  r.b = s.n * (int64_t)total;
+  return r;
+}
+
+// Checks shared by the variable-length entry points.  Returns FA_OK, a
+// negative status, or 1 when there is nothing to do.
+int check_varlen(int B, int H, int max_seqlen, int total, int d, float scale, int causal, float dropout_p,
+                 const int* cu_seqlens, const fa_strides* strides, int nstrides) {
+  int rc = check_common(B, H, max_seqlen, d, scale, causal, dropout_p);
+  if (rc != FA_OK) return rc;
+  if (total < 0) return FA_ERR_INVALID_ARG;
+  if (total == 0) return 1;
+  if ((long long)total * H * d > (1ll << 40)) return FA_ERR_TOO_LARGE;
+  if (!cu_seqlens || !strides) return FA_ERR_INVALID_ARG;
+  if (!aligned(cu_seqlens, 4)) return FA_ERR_ALIGNMENT;
+  for (int t = 0; t < nstrides; ++t) {
+    fa_strides s = strides[t];
+    s.b = 0;
+    if (!strides_ok(s)) return FA_ERR_ALIGNMENT;
+  }
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 200; }
 
 const char* fa_strerror(int status) {
   switch (status) {
@@ -224,6 +291,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   if ((rc = make_tile_map(&mk, k, B, H, N, d, strides[1])) != FA_OK) return rc;
   if ((rc = make_tile_map(&mv, v, B, H, N, d, strides[2])) != FA_OK) return rc;
   fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kv_hi = kAllTiles;
   a.B = B;
   a.H = H;
   a.N = N;
@@ -342,6 +411,7 @@ int bwd_setup(int B, int H, int N, int d, float scale, int causal, float dropout
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
   std::memset(a, 0, sizeof(*a));
+  a->kv_hi = kAllTiles;
   a->B = B;
   a->H = H;
   a->N = N;
@@ -350,7 +420,7 @@ int bwd_setup(int B, int H, int N, int d, float scale, int causal, float dropout
   a->drop_threshold = keep_threshold(dropout_p);
   a->drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
   a->seed = seed;
-  fa::bwd_workspace_split(workspace, B * H, N, d, &a->dq_acc, &a->lse2, &a->drow);
+  fa::bwd_workspace_split(workspace, B * H, N, d, &a->dq_acc, &a->lse2, &a->drow, &a->sched);
   a->err = device_error_ptr();
   if (!a->err) return cuda_fail(cudaErrorInvalidSymbol);
   return FA_OK;
@@ -548,6 +618,242 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   contiguous8(H, N, d, s);
   return fa_bwd_strided(q, k, v, o, dout, lse, dq, dk, dv, s, B, H, N, d, scale, causal, dropout_p, seed, workspace,
                         workspace_bytes, stream);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                  const int32_t* cu_seqlens, const int32_t* seqused, int B, int H, int max_seqlen, int total_tokens,
+                  int d, float scale, int causal, float dropout_p, uint64_t seed, void* stream) {
+  int rc = check_varlen(B, H, max_seqlen, total_tokens, d, scale, causal, dropout_p, cu_seqlens, strides, 4);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      (seqused && !aligned(seqused, 4)))
+    return FA_ERR_ALIGNMENT;
+  fa_strides s[4];
+  for (int t = 0; t < 4; ++t) s[t] = varlen_strides(strides[t], total_tokens);
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_tile_map(&mq, q, 1, H, total_tokens, d, s[0])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, 1, H, total_tokens, d, s[1])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, 1, H, total_tokens, d, s[2])) != FA_OK) return rc;
+  fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kv_hi = kAllTiles;
+  a.B = B;
+  a.H = H;
+  a.N = max_seqlen;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.drop_threshold = keep_threshold(dropout_p);
+  a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
+  a.seed = seed;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = 0;
+  a.o_sh = s[3].h;
+  a.o_sn = s[3].n;
+  a.lse = lse;
+  a.num_splits = 1;
+  a.cu_seqlens = cu_seqlens;
+  a.seqused = seqused;
+  a.total_tokens = total_tokens;
+  a.err = device_error_ptr();
+  if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool dropout = dropout_p > 0.f;
+  rc = d == 64 ? dispatch_fwd<64, fa::kFwdVarlen>(mq, mk, mv, a, causal != 0, dropout, st)
+               : dispatch_fwd<128, fa::kFwdVarlen>(mq, mk, mv, a, causal != 0, dropout, st);
+  if (rc != FA_OK || !seqused) return rc;
+  return launch_varlen_pad(B, H, max_seqlen, total_tokens, cu_seqlens, seqused, d, static_cast<__nv_bfloat16*>(o),
+                           s[3], nullptr, s[3], nullptr, s[3], lse, st);
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int H, int max_seqlen, int d) {
+  return fa_bwd_workspace_size(B, H, max_seqlen, d);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, const fa_strides* strides, const int32_t* cu_seqlens,
+                  const int32_t* seqused, int B, int H, int max_seqlen, int total_tokens, int d, float scale,
+                  int causal, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int rc = check_varlen(B, H, max_seqlen, total_tokens, d, scale, causal, dropout_p, cu_seqlens, strides, 8);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) ||
+      (seqused && !aligned(seqused, 4)))
+    return FA_ERR_ALIGNMENT;
+  fa::BwdArgs a;
+  if ((rc = bwd_setup(B, H, max_seqlen, d, scale, causal, dropout_p, seed, workspace, workspace_bytes, &a)) !=
+      FA_OK)
+    return rc;
+  fa_strides s[8];
+  for (int t = 0; t < 8; ++t) s[t] = varlen_strides(strides[t], total_tokens);
+  a.cu_seqlens = cu_seqlens;
+  a.seqused = seqused;
+  a.total_tokens = total_tokens;
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.o_sh = s[3].h;
+  a.o_sn = s[3].n;
+  a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.do_sh = s[4].h;
+  a.do_sn = s[4].n;
+  a.lse = lse;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dq_sh = s[5].h;
+  a.dq_sn = s[5].n;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dk_sh = s[6].h;
+  a.dk_sn = s[6].n;
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dv_sh = s[7].h;
+  a.dv_sn = s[7].n;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((rc = make_tile_map(&mq, q, 1, H, total_tokens, d, s[0])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, 1, H, total_tokens, d, s[1])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, 1, H, total_tokens, d, s[2])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mdo, dout, 1, H, total_tokens, d, s[4])) != FA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fa::launch_bwd_prepare(a, d, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_bwd_recompute(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = fa::launch_bwd_finalize(a, d, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!seqused) return FA_OK;
+  return launch_varlen_pad(B, H, max_seqlen, total_tokens, cu_seqlens, seqused, d, static_cast<__nv_bfloat16*>(dq),
+                           s[5], static_cast<__nv_bfloat16*>(dk), s[6], static_cast<__nv_bfloat16*>(dv), s[7],
+                           nullptr, st);
+}
+
+namespace {
+
+// A key window [kv_begin, kv_end) of an N-key sequence: kv_begin a multiple
+// of the 128-key tile, kv_end a multiple of it or N.
+bool key_window_ok(int N, int kv_begin, int kv_end) {
+  return 0 <= kv_begin && kv_begin <= kv_end && kv_end <= N && kv_begin % 128 == 0 &&
+         (kv_end == N || kv_end % 128 == 0);
+}
+
+}  // namespace
+
+int fa_fwd_partial(const void* q, const void* k, const void* v, float* part_o, float* part_lse, int B, int H, int N,
+                   int d, float scale, int causal, float dropout_p, uint64_t seed, int kv_begin, int kv_end,
+                   void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!key_window_ok(N, kv_begin, kv_end)) return FA_ERR_INVALID_ARG;
+  const int nk = kv_end - kv_begin;
+  if (!q || !part_o || !part_lse || (nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(part_o, 16) || !aligned(part_lse, 4) ||
+      (nk > 0 && (!aligned(k, 16) || !aligned(v, 16))))
+    return FA_ERR_ALIGNMENT;
+  CUtensorMap mq, mk, mv;
+  if ((rc = make_tile_map(&mq, q, B, H, N, d, contiguous_strides(H, N, d))) != FA_OK) return rc;
+  // an empty window reads no key: its maps only need to be valid
+  const void* kb = nk > 0 ? k : q;
+  const void* vb = nk > 0 ? v : q;
+  const int nkm = nk > 0 ? nk : N;
+  if ((rc = make_tile_map(&mk, kb, B, H, nkm, d, contiguous_strides(H, nkm, d))) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, vb, B, H, nkm, d, contiguous_strides(H, nkm, d))) != FA_OK) return rc;
+  fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.drop_threshold = keep_threshold(dropout_p);
+  a.drop_scale = (float)(1.0 / (1.0 - (double)dropout_p));
+  a.seed = seed;
+  a.num_splits = 1;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.kv_lo = kv_begin / 128;
+  a.kv_hi = nk > 0 ? (kv_end + 127) / 128 : kv_begin / 128;
+  a.kv_row_off = kv_begin;
+  a.partial_only = 1;
+  a.err = device_error_ptr();
+  if (!a.err) return cuda_fail(cudaErrorInvalidSymbol);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool dropout = dropout_p > 0.f;
+  return d == 64 ? dispatch_fwd<64, fa::kFwdSplit>(mq, mk, mv, a, causal != 0, dropout, st)
+                 : dispatch_fwd<128, fa::kFwdSplit>(mq, mk, mv, a, causal != 0, dropout, st);
+}
+
+int fa_merge_partials(const float* part_o, const float* part_lse, int num_parts, void* o, float* lse, int B, int H,
+                      int N, int d, void* stream) {
+  int rc = check_common(B, H, N, d, 1.f, 0, 0.f);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (num_parts < 1 || num_parts > 4096) return FA_ERR_INVALID_ARG;
+  if (!part_o || !part_lse || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(part_o, 16) || !aligned(o, 16) || !aligned(part_lse, 4) || !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  const fa_strides s = contiguous_strides(H, N, d);
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_sb = s.b;
+  a.o_sh = s.h;
+  a.o_sn = s.n;
+  a.lse = lse;
+  a.num_splits = num_parts;
+  a.part_o = const_cast<float*>(part_o);
+  a.part_lse = const_cast<float*>(part_lse);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fa::splitkv_combine_kernel<64><<<148 * 8, 256, 0, st>>>(a);
+  else
+    fa::splitkv_combine_kernel<128><<<148 * 8, 256, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+size_t fa_bwd_dq_accumulator_bytes(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.f, 0, 0.f) != FA_OK) return 0;
+  return fa::round_up((size_t)B * H * fa::round_up((size_t)N, 128) * d * 4, 256);
+}
+
+int fa_bwd_recompute_range(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
+                           int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int kv_begin,
+                           int kv_end, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(B, H, N, d, scale, causal, dropout_p);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!key_window_ok(N, kv_begin, kv_end)) return FA_ERR_INVALID_ARG;
+  const int nk = kv_end - kv_begin;
+  if (nk == 0) return FA_OK;  // no key of this window: nothing to add
+  if (!q || !k || !v || !dout || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16))
+    return FA_ERR_ALIGNMENT;
+  fa::BwdArgs a;
+  if ((rc = bwd_setup(B, H, N, d, scale, causal, dropout_p, seed, workspace, workspace_bytes, &a)) != FA_OK)
+    return rc;
+  const fa_strides sk = contiguous_strides(H, nk, d);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dk_sb = sk.b;
+  a.dk_sh = sk.h;
+  a.dk_sn = sk.n;
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dv_sb = sk.b;
+  a.dv_sh = sk.h;
+  a.dv_sn = sk.n;
+  a.kv_lo = kv_begin / 128;
+  a.kv_hi = (kv_end + 127) / 128;
+  a.kv_row_off = kv_begin;
+  CUtensorMap mq, mk, mv, mdo;
+  const fa_strides sq = contiguous_strides(H, N, d);
+  if ((rc = make_tile_map(&mq, q, B, H, N, d, sq)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B, H, nk, d, sk)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B, H, nk, d, sk)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mdo, dout, B, H, N, d, sq)) != FA_OK) return rc;
+  cudaError_t e = fa::launch_bwd_recompute(mq, mk, mv, mdo, a, d, causal != 0, dropout_p > 0.f,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 }  // extern "C"

@@ -31,6 +31,14 @@
 // the MMA issuer skips the products of a tile its query tile does not see.
 // A query tile that sees no key tile writes O = 0 and lse = -inf.
 //
+// Variable-length mode ("FlashAttention for Efficient Training" section 5.2,
+// Handling Variable Sequence Lengths): the B sequences are stored token-major
+// and sequence b owns tokens [cu_seqlens[b], cu_seqlens[b+1]), of which the
+// first L_b are real (seqused[b], else all of them).  A CTA covers 256 rows of
+// one sequence and head; keys at or beyond L_b are masked like the ragged
+// last tile of a dense problem, and a CTA whose rows all lie at or beyond L_b
+// returns at once, so no work is spent on padding.
+//
 // Online softmax in base 2: x = s * scale * log2(e); m is a running row
 // maximum that is only raised (and O, l rescaled) when the tile maximum
 // exceeds it by more than 8, i.e. a factor 256.  Every P and l use the same
@@ -58,6 +66,10 @@ struct FwdArgs {
   int num_splits;
   float* part_o;
   float* part_lse;
+  // split-KV key window: only key tiles [kv_lo, kv_hi) are split (and seen);
+  // the K/V tensors hold key rows from kv_row_off on (a rank's key chunk)
+  int kv_lo, kv_hi, kv_row_off;
+  int partial_only;  // host side: split-KV pieces are the output (no combine pass)
   // block-sparse (SPARSE kernels only): bmask[hm][qt][kt] != 0 lets query
   // tile qt see key tile kt; hm = 0 when bmask_heads == 1, else the head
   const uint8_t* bmask;
@@ -65,10 +77,16 @@ struct FwdArgs {
   // fault injection for tests: the producer issues no K/V load, so the MMA
   // warp's first wait runs out and the kernel reports a timeout
   int debug_skip_kv;
+  // variable-length (VARLEN kernels only): token offsets [B+1], optional used
+  // lengths [B], the token count T (q/k/v/o rows; lse is [H, T]); N holds the
+  // largest slot size and sizes the grid
+  const int* cu_seqlens;
+  const int* seqused;
+  int total_tokens;
 };
 
-// Kernel variants: plain, split-KV, block-sparse.
-enum FwdMode : int { kFwdPlain = 0, kFwdSplit = 1, kFwdSparse = 2 };
+// Kernel variants: plain, split-KV, block-sparse, variable-length.
+enum FwdMode : int { kFwdPlain = 0, kFwdSplit = 1, kFwdSparse = 2, kFwdVarlen = 3 };
 
 // Of every 8 pairs of probabilities, this many take the exponential on the
 // FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
@@ -99,6 +117,7 @@ __global__ void __launch_bounds__(320, 1)
   using L = FwdLayout<D>;
   constexpr bool SPLIT = MODE == kFwdSplit;
   constexpr bool SPARSE = MODE == kFwdSparse;
+  constexpr bool VARLEN = MODE == kFwdVarlen;
   static_assert(D == 64 || D == 128, "head dim");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -129,9 +148,21 @@ __global__ void __launch_bounds__(320, 1)
   const int bh = work - tile_rev * BH;
   const int cta_tile = CAUSAL ? (n_cta_tiles - 1 - tile_rev) : tile_rev;
   const int bb = bh / a.H, hh = bh - bb * a.H;  // batch and head of this CTA
-  const int n_kv_all = (a.N + 127) >> 7;
+  // this CTA's sequence: real rows [0, seq_len) at tokens row0.. of the
+  // tensors, batch coordinate wc of the tensor maps
+  int seq_len = a.N, row0 = 0, wc = bb;
+  long long lse_base = (long long)bh * a.N;
+  if (VARLEN) {
+    const SeqSpan sp = varlen_span(a.cu_seqlens, a.seqused, bb, a.total_tokens, a.N, a.err, cta_tile == 0);
+    seq_len = sp.len;
+    row0 = sp.row0;
+    wc = 0;
+    lse_base = (long long)hh * a.total_tokens + row0;
+    if (cta_tile * 256 >= seq_len) return;  // only padding (or nothing) here: no work
+  }
+  const int n_kv_all = (seq_len + 127) >> 7;
   const int qt0 = 2 * cta_tile;
-  const bool act1 = (qt0 + 1) * 128 < a.N;
+  const bool act1 = (qt0 + 1) * 128 < seq_len;
   // key tiles each Q tile sees: [0, end_t)
   const int end0 = CAUSAL ? qt0 + 1 : n_kv_all;
   const int end1 = act1 ? (CAUSAL ? qt0 + 2 : n_kv_all) : 0;
@@ -140,9 +171,10 @@ __global__ void __launch_bounds__(320, 1)
   // tile t processes here, local index jj = j - j0 drives the pipelines
   int j0 = 0, span = end_max;
   if (SPLIT) {
-    const int chunk = (end_max + a.num_splits - 1) / a.num_splits;
-    j0 = split * chunk;
-    span = max(0, min(end_max, j0 + chunk) - j0);
+    const int hi = min(a.kv_hi, end_max), lo = min(a.kv_lo, hi);
+    const int chunk = (hi - lo + a.num_splits - 1) / a.num_splits;
+    j0 = lo + split * chunk;
+    span = max(0, min(hi, j0 + chunk) - j0);
   }
   // steps of the K/V stream (nkv_max) and how many of them each Q tile uses
   int nkv0 = max(0, min(end0, j0 + span) - j0);
@@ -211,8 +243,8 @@ __global__ void __launch_bounds__(320, 1)
         if (t == 1 && !act1) break;
         mbar_arrive_expect_tx(&bar_q[t], L::kTile);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, (qt0 + t) * 128, hh, bb,
-                      &bar_q[t], pol_once);
+          tma_load_4d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, row0 + (qt0 + t) * 128, hh,
+                      wc, &bar_q[t], pol_once);
       }
       int stage = 0;
       uint32_t phase = 0;
@@ -229,8 +261,8 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h, kt * 128, hh, bb,
-                        &bar_kv_full[stage], pol_keep);
+            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h,
+                        row0 + kt * 128 - a.kv_row_off, hh, wc, &bar_kv_full[stage], pol_keep);
           ++issued;
           if (++stage == L::kStages) {
             stage = 0;
@@ -387,7 +419,7 @@ __global__ void __launch_bounds__(320, 1)
         // only the diagonal tile (causal) or the ragged last tile masks
         int lim = 128;
         if (CAUSAL && jg == qt0 + t) lim = r + 1;
-        if (!CAUSAL && jg == n_kv_all - 1 && (a.N & 127)) lim = a.N - jg * 128;
+        if (!CAUSAL && jg == n_kv_all - 1 && (seq_len & 127)) lim = seq_len - jg * 128;
         if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -487,14 +519,14 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(&bar_p[t]);
       }
       // epilogue: O = O_t / l, lse = (m + log2 l) ln 2
-      const bool in_range = q_row < a.N;
+      const bool in_range = q_row < seq_len;
       if (SPARSE && nkv == 0) {
         // the mask hides every key tile from this query tile
         if (in_range && ok) {
           __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)q_row * a.o_sn;
 #pragma unroll
           for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
-          a.lse[(size_t)bh * a.N + q_row] = -INFINITY;
+          a.lse[lse_base + q_row] = -INFINITY;
         }
       } else if (SPLIT && nkv == 0) {
         // this split holds no key tile of this query tile: an empty partial
@@ -524,7 +556,8 @@ __global__ void __launch_bounds__(320, 1)
           }
           if (in_range) a.part_lse[((size_t)split * BH + bh) * a.N + q_row] = lse_row;
         } else {
-          __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)(in_range ? q_row : 0) * a.o_sn;
+          __nv_bfloat16* orow =
+              a.o + bb * a.o_sb + hh * a.o_sh + (long long)(row0 + (in_range ? q_row : 0)) * a.o_sn;
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t o[32];
@@ -539,7 +572,7 @@ __global__ void __launch_bounds__(320, 1)
                 st_global_v4(orow + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
             }
           }
-          if (in_range) a.lse[(size_t)bh * a.N + q_row] = lse_row;
+          if (in_range) a.lse[lse_base + q_row] = lse_row;
         }
       }
     }

@@ -17,6 +17,7 @@ enum : int {
   kDevOk = 0,
   kDevTimeout = 1,      // a bounded mbarrier wait ran out
   kDevMisaligned = 2,   // shared-memory tile base not 1024-byte aligned
+  kDevBadSeqlens = 3,   // variable-length offsets or lengths out of range (clamped)
 };
 
 // Upper bound on any single wait (ns).  Kernels here run for milliseconds;
@@ -436,6 +437,33 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
   return v;
+}
+
+// ------------------------------------------------ variable-length batches
+
+// Where sequence b of a variable-length batch lives: its first token, its slot
+// size and its real length.  Offsets are clamped into [0, T] and lengths into
+// the slot and into max_slot, so every row index derived from them stays
+// inside the caller's tensors even if the offsets are inconsistent; an
+// inconsistency is also recorded in the device error word.
+struct SeqSpan {
+  int row0, slot, len;
+};
+
+__device__ __forceinline__ SeqSpan varlen_span(const int* cu, const int* used, int b, int total, int max_slot,
+                                               int* err, bool report) {
+  int s0 = __ldg(cu + b), s1 = __ldg(cu + b + 1);
+  const bool bad = s0 < 0 || s1 < s0 || s1 > total || s1 - s0 > max_slot;
+  s0 = min(max(s0, 0), total);
+  s1 = min(max(s1, s0), total);
+  SeqSpan r;
+  r.row0 = s0;
+  r.slot = min(s1 - s0, max_slot);
+  int L = used ? __ldg(used + b) : r.slot;
+  const bool bad_used = used && (L < 0 || L > r.slot);
+  r.len = min(max(L, 0), r.slot);
+  if (report && (bad || bad_used) && err) atomicCAS(err, kDevOk, kDevBadSeqlens);
+  return r;
 }
 
 // ---------------------------------------------------- block-sparse tile sets

@@ -30,3 +30,23 @@ def max_over_ranks(values, device=None) -> list:
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.tolist()]
+
+
+def all_ranks_ok(ok: bool, device=None) -> bool:
+    """True on every rank iff ``ok`` holds on every rank (identity when
+    torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([1.0 if ok else 0.0], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item() > 0.5)
+
+
+def replica_summary(elapsed_ms: float, e2e_ms: float, stage_ms: list, ok: bool, device=None) -> dict:
+    """What one job reports from its replicas: the slowest rank's timings
+    (the job is done when the last replica is) and whether every replica's
+    output passed its checks.  Every rank takes the same collective steps."""
+    times = max_over_ranks([elapsed_ms, e2e_ms] + list(stage_ms), device=device)
+    return {"elapsed_ms": times[0], "e2e_ms": times[1], "stage_ms": times[2:],
+            "all_ok": all_ranks_ok(ok, device=device)}

@@ -1,0 +1,105 @@
+"""Sequence parallelism across GPUs for long sequences.
+
+"FlashAttention for Efficient Training", section 5.3 (Sequence Parallelism
+for Long Contexts): the sequence is cut into chunks held by different GPUs,
+and the output for a query needs every key chunk.  The page's formula sums a
+softmax per key chunk; read exactly, the output is the logsumexp merge of the
+softmax pieces over the chunks -- the same identity as the online softmax and
+the split-KV merge (section 6.1).
+
+Layout: every rank holds the queries and dO of the whole sequence (q, do
+dense [B, H, N, d]) and one window of the keys (k, v dense [B, H, Nk, d],
+key rows [kv_begin, kv_begin + Nk)), the windows of the ranks tiling the
+sequence in rank order (``key_windows``).
+
+  forward:  each rank computes the softmax piece of every query over its
+            keys (``fa_fwd_partial``: O_r normalised over its keys, lse_r);
+            the pieces are all-gathered (NCCL) and every rank merges them
+            (``fa_merge_partials``) into the full O and lse.
+  backward: each rank forms D = dO . O and the scaled lse from the full O
+            (``fa_bwd_prepare``), recomputes its key window
+            (``fa_bwd_recompute_range``: its dK, dV complete, its part of dQ
+            into the fp32 accumulator), the accumulators are summed over the
+            ranks (NCCL all-reduce), and ``fa_bwd_finalize`` converts dQ.
+
+The exchanges are the only collectives; the compute steps come from an ops
+object (``CudaOps`` on GPUs), so the same orchestration runs under a CPU
+test double in multi-process tests.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+TILE = 128
+
+
+def key_windows(N: int, world: int) -> list:
+    """Key windows [(begin, end)] of the ranks: the ceil(N / 128) key tiles
+    split as evenly as possible, in rank order (a rank may get none)."""
+    if world < 1 or N < 0:
+        raise ValueError("bad world size or length")
+    nt = (N + TILE - 1) // TILE
+    out = []
+    for r in range(world):
+        t0, t1 = r * nt // world, (r + 1) * nt // world
+        out.append((min(t0 * TILE, N), min(t1 * TILE, N)))
+    return out
+
+
+class CudaOps:
+    """The per-rank compute steps on the GPU, through the C ABI."""
+
+    def __init__(self):
+        from io_aware_exact_25_b200 import binding
+        self.b = binding
+
+    def fwd_partial(self, q, k, v, kv_begin, causal, scale, dropout_p, seed):
+        return self.b.fwd_partial(q, k, v, kv_begin, causal=causal, scale=scale, dropout_p=dropout_p, seed=seed)
+
+    def merge(self, part_o, part_lse):
+        return self.b.merge_partials(part_o, part_lse)
+
+    def bwd_begin(self, o, do, lse):
+        B, H, N, d = o.shape
+        ws = torch.empty(self.b.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=o.device)
+        self.b.bwd_prepare(o, do, lse, ws)
+        return ws
+
+    def bwd_range(self, ws, q, k, v, do, kv_begin, causal, scale, dropout_p, seed):
+        return self.b.bwd_recompute_range(q, k, v, do, kv_begin, ws, causal=causal, scale=scale,
+                                          dropout_p=dropout_p, seed=seed)
+
+    def dq_accumulator(self, ws, q):
+        B, H, N, d = q.shape
+        return ws[: self.b.dq_accumulator_bytes(B, H, N, d)].view(torch.float32)
+
+    def bwd_end(self, ws, q, scale):
+        return self.b.bwd_finalize(torch.empty_like(q), ws, scale)
+
+
+def forward(q, k, v, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, group=None, ops=None):
+    """Full O and lse on every rank from the ranks' key windows."""
+    ops = ops or CudaOps()
+    d = q.shape[-1]
+    scale = scale if scale is not None else d ** -0.5
+    part_o, part_lse = ops.fwd_partial(q, k, v, kv_begin, causal, scale, dropout_p, seed)
+    world = dist.get_world_size(group)
+    gathered = []
+    for t in (part_o, part_lse):
+        flat = torch.empty(world * t.numel(), dtype=t.dtype, device=t.device)
+        dist.all_gather_into_tensor(flat, t.contiguous().view(-1), group=group)
+        gathered.append(flat.view((world,) + tuple(t.shape)))
+    return ops.merge(*gathered)
+
+
+def backward(q, k, v, o, do, lse, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, group=None, ops=None):
+    """dQ (full, on every rank) and dK, dV of this rank's key window."""
+    ops = ops or CudaOps()
+    d = q.shape[-1]
+    scale = scale if scale is not None else d ** -0.5
+    ws = ops.bwd_begin(o, do, lse)
+    dk, dv = ops.bwd_range(ws, q, k, v, do, kv_begin, causal, scale, dropout_p, seed)
+    dist.all_reduce(ops.dq_accumulator(ws, q), op=dist.ReduceOp.SUM, group=group)
+    dq = ops.bwd_end(ws, q, scale)
+    return dq, dk, dv

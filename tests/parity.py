@@ -15,8 +15,11 @@ an element with |ref| >= 4 may exceed 2e-2 by up to
     half_ulp(|ref|) + (2e-2 - 2^-7),
 and no more.  Every element that uses the exception is counted: ``check``
 records, per call, how many elements lie in (2e-2, that bound] and the worst
-one; the count may not exceed ``max(4, 1e-4 * elements)`` (so a systematic
-error cannot hide behind it); and the session prints every such record at
+one.  The count may not exceed ``max(4, 1e-4 * elements)`` plus the number of
+elements with |ref| >= 8, where half an ulp (2^-5 and up) exceeds 2e-2 by
+itself and a large share of correctly rounded outputs lies above it; in
+[4, 8) only an error of more than 2e-2 - 2^-6 before the rounding gets there,
+so a systematic error cannot hide behind the exception.  The session prints every such record at
 the end (``tests/conftest.py``), and writes them as JSON lines to the file
 ``FA_PARITY_REPORT`` names, if that variable is set.
 """
@@ -86,7 +89,7 @@ def check(name, got, ref, exclude_rows=None, scale: float = 1.0):
     n_over = int(over.sum())
     if n_over:
         w = np.unravel_index(np.argmax(np.where(over, err, 0.0)), err.shape)
-        cap = max(EXC_FLOOR, int(EXC_FRACTION * err.size))
+        cap = max(EXC_FLOOR, int(EXC_FRACTION * err.size)) + int((np.abs(ref) >= 8.0 * scale).sum())
         _record({"test": _current_test["id"], "tensor": name, "elements": int(err.size), "over_2e-2": n_over,
                  "cap": cap, "worst_err": float(err[w]), "ref_at_worst": float(ref[w]),
                  "bound_at_worst": float(bound[w]), "scale": scale})

