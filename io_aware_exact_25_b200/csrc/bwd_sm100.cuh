@@ -283,6 +283,9 @@ struct BwdLayout {
 // two P/dS warpgroups: queries 0-63 at [0,32), 64-127 at [64,96).
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
 
+// Visit each work item's query tiles from a rotated start (see q_tile).
+constexpr bool kRotateQueryTiles = true;
+
 // Of every 8 pairs of recomputed probabilities, this many take the
 // exponential on the FMA pipe (polynomial), the rest on MUFU.
 constexpr int kBwdPolyPairsOf8 = 0;
@@ -353,7 +356,7 @@ __global__ void __launch_bounds__(448, 1)
   // An item's sequence: real rows [0, len) at tokens row0.. of the tensors,
   // batch coordinate wc of the tensor maps (variable-length: 0).
   struct Item {
-    int jt, bh, bb, hh, i_begin, n_steps, row0, len, wc;
+    int jt, bh, bb, hh, i_begin, n_steps, row0, len, wc, rot;
   };
   auto item_of = [&](int w) {
     const int grp = min(w / (hg * nTr), n_groups - 1);
@@ -379,7 +382,18 @@ __global__ void __launch_bounds__(448, 1)
       const int nTb = (sp.len + 127) >> 7;
       t.n_steps = t.jt < nTb ? nTb - t.i_begin : 0;
     }
+    // The item visits its query tiles starting at a rotation of its own, so
+    // items of one head that run at the same time reduce their dQ partials
+    // into different accumulator tiles instead of all into the same one.
+    t.rot = t.n_steps > 1 ? (int)(((uint32_t)t.jt * 2654435761u + (uint32_t)t.bh * 40503u) % (uint32_t)t.n_steps) : 0;
     return t;
+  };
+  // query tile of step `it` of item t (dense items; block-sparse ones walk
+  // their bit set in order)
+  auto q_tile = [&](const Item& t, int it) {
+    int s = it + (kRotateQueryTiles ? t.rot : 0);
+    if (s >= t.n_steps) s -= t.n_steps;
+    return t.i_begin + s;
   };
   uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // SPARSE: query tiles that see jt
   int* sparse_cnt = reinterpret_cast<int*>(qbits + kSparseWords);
@@ -513,7 +527,7 @@ __global__ void __launch_bounds__(448, 1)
       BitWalk walk(qbits, qbits, nwords);
       for (int it = 0; it < t.n_steps; ++it) {
         const int gs = g + it;
-        const int i = SPARSE ? walk.next() : t.i_begin + it;
+        const int i = SPARSE ? walk.next() : q_tile(t, it);
         // Q_i and dO_i: re-read by every key tile of the head -> keep in L2
         const int qs = gs & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar_q_empty[qs], ((gs >> 1) & 1) ^ 1u, ab))) {
@@ -751,7 +765,7 @@ __global__ void __launch_bounds__(448, 1)
     const Item t = item_at(w);
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
-      const int i = SPARSE ? walk.next() : t.i_begin + it;
+      const int i = SPARSE ? walk.next() : q_tile(t, it);
       // the staging tiles are free once the previous step's reductions read them
       if (leader) {
         bulk_wait_read<0>();
@@ -837,7 +851,7 @@ __global__ void __launch_bounds__(448, 1)
     const bool key_ok = key < t.len;
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
-      const int i = SPARSE ? walk.next() : t.i_begin + it;
+      const int i = SPARSE ? walk.next() : q_tile(t, it);
       const int gs = g + it;
       const uint32_t ph = gs & 1;
       const int rs = gs % L::kRowStages;
