@@ -24,8 +24,8 @@
 //     S^T = K_j Q_i^T and dP^T = V_j dO_i^T, forms P^T and dS^T in registers,
 //     accumulates dV += P^T dO_i (P^T from tensor memory) and dK += dS^T Q_i
 //     (dS from shared memory) in tensor memory, and
-//     computes the dQ_i partial dS K_j, which a warpgroup stages in shared
-//     memory and adds into the fp32 accumulator with bulk reductions;
+//     computes the dQ_i partial dS K_j, which a warpgroup adds into the fp32
+//     accumulator from registers with vector reductions;
 //  3. dQ = scale * accumulator, rounded to bf16.
 // Variable-length mode ("FlashAttention for Efficient Training" section 5.2):
 // sequences stored token-major at offsets cu_seqlens; a CTA's item is a key
@@ -101,10 +101,12 @@ struct BwdArgs {
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace: the fp32 dQ accumulator over N rounded up to 128 rows, stored
-// tile by tile -- for each head, 128-row query tile and 16-column piece, one
-// contiguous 8 KB block of 128 rows x 16 columns whose 16-byte chunks are
-// permuted by the 64-byte swizzle (chunk k of row r at k ^ ((r >> 1) & 3)) --
-// then the scaled lse and D row vectors, then the item counter.
+// tile by tile -- for each head and 128-row query tile one contiguous block of
+// 128 x D floats.  At d = 64 the block is chunk-major: the four columns
+// 4c..4c+3 of row r at (c * 128 + r) * 4.  At d = 128 it is eight 16-column
+// pieces of 8 KB, each 128 rows x 16 columns with its 16-byte chunks permuted
+// by the 64-byte swizzle (chunk k of row r at k ^ ((r >> 1) & 3)).  Then the
+// scaled lse and D row vectors, then the item counter.
 inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   const size_t npad = round_up((size_t)N, 128);
   return round_up((size_t)BH * npad * d * 4, 256) + 2 * round_up((size_t)BH * npad * 4, 256) + 256;
@@ -198,35 +200,63 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
     acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ = scale * accumulator, read from the tiled accumulator layout; each
-// thread converts 8 consecutive columns (two swizzled 16-byte chunks) of a row.
+// dQ = scale * accumulator.  Each thread converts 8 columns (two 4-column
+// chunks) of one row.  d = 64 (chunk-major tiles): a warp takes 32
+// consecutive rows of one chunk pair, so its reads are two contiguous
+// 512-byte runs.  d = 128 (swizzled 16-column pieces): consecutive threads
+// take consecutive chunk pairs of one row, so its writes are contiguous.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                        int BH, int H, int N, long long sb, long long sh, long long sn,
                                                        float scale, const int* cu_seqlens, const int* seqused,
                                                        int total_tokens) {
-  const int npad = (N + 127) & ~127;
-  const long long n8 = (long long)BH * N * (D / 8);
-  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n8;
+  constexpr bool kChunkMajor = D == 64;
+  const int nT = (N + 127) >> 7;
+  constexpr int kC8 = D / 8;  // chunk pairs per row
+  const long long n = (long long)BH * nT * 128 * kC8;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n;
        u += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(u % (D / 8));
-    const long long rowg = u / (D / 8);
-    const int bh = (int)(rowg / N);
-    const int i = (int)(rowg - (long long)bh * N);
-    const int tile = i >> 7, r = i & 127;
-    const int piece = c8 >> 1;            // 16-column piece
-    const int k0 = (c8 & 1) * 2;          // first of the two 4-column chunks
-    const int sw = (r >> 1) & 3;
+    int c8, r, tile, bh;
+    if (kChunkMajor) {  // (bh, tile, row group, chunk pair, lane)
+      const int j = (int)(u & 31);
+      long long v = u >> 5;
+      c8 = (int)(v % kC8);
+      v /= kC8;
+      r = (int)(v & 3) * 32 + j;
+      v >>= 2;
+      tile = (int)(v % nT);
+      bh = (int)(v / nT);
+    } else {  // (bh, tile, row, chunk pair)
+      c8 = (int)(u % kC8);
+      long long v = u / kC8;
+      r = (int)(v & 127);
+      v >>= 7;
+      tile = (int)(v % nT);
+      bh = (int)(v / nT);
+    }
+    const int i = tile * 128 + r;
     const int b_ = bh / H, h_ = bh - b_ * H;
     long long row = i;
+    int len = N;
     if (cu_seqlens) {
       const SeqSpan sp = varlen_span(cu_seqlens, seqused, b_, total_tokens, N, nullptr, false);
-      if (i >= sp.len) continue;  // padding rows are filled separately
+      len = sp.len;  // padding rows are filled separately
       row = sp.row0 + i;
     }
-    const float* blk = acc + (((size_t)bh * (npad >> 7) + tile) * (D / 16) + piece) * 2048 + r * 16;
-    const float4 x = *reinterpret_cast<const float4*>(blk + ((k0 ^ sw) << 2));
-    const float4 y = *reinterpret_cast<const float4*>(blk + (((k0 + 1) ^ sw) << 2));
+    if (i >= len) continue;
+    const float* blk = acc + ((size_t)bh * nT + tile) * (size_t)(128 * D);
+    float4 x, y;
+    if (kChunkMajor) {
+      x = *reinterpret_cast<const float4*>(blk + ((2 * c8) * 128 + r) * 4);
+      y = *reinterpret_cast<const float4*>(blk + ((2 * c8 + 1) * 128 + r) * 4);
+    } else {
+      const int piece = c8 >> 1;    // 16-column piece
+      const int k0 = (c8 & 1) * 2;  // first of the two 4-column chunks
+      const int sw = (r >> 1) & 3;
+      const float* pr = blk + piece * 2048 + r * 16;
+      x = *reinterpret_cast<const float4*>(pr + ((k0 ^ sw) << 2));
+      y = *reinterpret_cast<const float4*>(pr + (((k0 + 1) ^ sw) << 2));
+    }
     uint4 w;
     w.x = pack_bf16x2(x.x * scale, x.y * scale);
     w.y = pack_bf16x2(x.z * scale, x.w * scale);
@@ -254,10 +284,14 @@ struct BwdLayout {
   // double-buffered row statistics, except where shared memory runs out
   static constexpr int kRowStages = (D == 128 && DROPOUT) ? 1 : 2;
   static constexpr uint32_t kOffRow = kOffDS + 2u * kHalf;
-  // dQ staging: 128-row x 16-column fp32 pieces (64-byte rows, 64-byte
-  // swizzle), each the source of one 8 KB bulk reduction
+  // dQ accumulation: at d = 64 straight from registers (vector reductions);
+  // at d = 128 through shared memory: 128-row x 16-column fp32 pieces
+  // (64-byte rows, 64-byte swizzle), each the source of one 8 KB bulk
+  // reduction (measured: direct reductions win 4% at d = 64 and lose 1% at
+  // d = 128, where they also make the dQ conversion's writes strided)
+  static constexpr bool kDqDirect = D == 64;
   static constexpr uint32_t kDqPiece = 128u * 64u;
-  static constexpr int kDqBufs = 4;
+  static constexpr int kDqBufs = kDqDirect ? 0 : 4;
   static constexpr uint32_t kOffDQ = (kOffRow + kRowStages * kRowStage + 1023u) & ~1023u;
   static constexpr uint32_t kOffBar = kOffDQ + kDqBufs * kDqPiece;
   // kv, q_full[2], q_empty[2], do_full[2], do_empty[2], row_full[2],
@@ -265,7 +299,7 @@ struct BwdLayout {
   // item_full[2], item_empty[2]
   static constexpr int kNumBars = 1 + 12 + 10 + 4;
   // after the barriers: TMEM address, abort flag, dQ-warpgroup flag, two item
-  // slots, the dQ warpgroup's item
+  // slots
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 32;
   // block-sparse: the query-tile bit set and its count after the barriers
   static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
@@ -284,7 +318,9 @@ struct BwdLayout {
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
 
 // Visit each work item's query tiles from a rotated start (see q_tile).
-constexpr bool kRotateQueryTiles = true;
+// Measured within noise (+1.3% on long8k, -1% on train2k) and it changes the
+// dK/dV summation order against the one-item-per-CTA kernels; off.
+constexpr bool kRotateQueryTiles = false;
 
 // Of every 8 pairs of recomputed probabilities, this many take the
 // exponential on the FMA pipe (polynomial), the rest on MUFU.
@@ -320,11 +356,10 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* bar_drain = bars + 21;
   uint64_t* bar_acc_free = bars + 22;  // dV/dK accumulators read out by the epilogue
   uint64_t* bar_item_full = bars + 23;   // [2] the producer published the next item
-  uint64_t* bar_item_empty = bars + 25;  // [2] every role has read it (10 arrivals)
+  uint64_t* bar_item_empty = bars + 25;  // [2] every role has read it (13 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);  // [0] abort, [1] dQ warpgroup flag
   int* item_slot = abort_flag + 2;                           // [2] published item indices
-  int* dq_item = abort_flag + 4;                             // the dQ warpgroup's current item
   const uint32_t sbase = smem_u32(smem);
 
   const int BH = a.B * a.H;
@@ -421,7 +456,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_drain, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_item_full[s], 1);
-      mbar_init(&bar_item_empty[s], 10);  // MMA thread, dQ leader, 8 P/dS warps
+      mbar_init(&bar_item_empty[s], 13);  // MMA thread, 4 dQ warps, 8 P/dS warps
     }
     const bool misaligned = (sbase & 1023u) != 0u;
     *abort_flag = misaligned ? 1 : 0;
@@ -710,22 +745,33 @@ __global__ void __launch_bounds__(448, 1)
   } else if (run && warp >= 8 && warp < 12) {
     // ------------------------------------------ dQ read-out + accumulate
     // The partial dQ_i (128 rows x D fp32, query rows on the TMEM lanes) is
-    // added into the fp32 accumulator in 16-column pieces: every thread
-    // writes its row of a piece into a 64-byte-swizzled staging tile, and
-    // one thread adds each whole 8 KB tile with a bulk reduction.  With four
-    // staging tiles, the first 64 columns are staged while the rest is still
-    // being read from TMEM; the TMEM columns are released as soon as the whole
-    // row is in registers or shared memory, before any reduction waits.  The
-    // loop is uniform over the warpgroup (one thread waits, a named barrier
-    // shares the outcome), so every thread reaches every named barrier.
-    static_assert(D == 64 || L::kDqBufs >= 4, "staging tiles");
+    // added into the fp32 accumulator.  At d = 64 straight from registers
+    // with vector reductions (red.global.add.v4.f32), each warp instruction
+    // covering 512 contiguous bytes of the chunk-major accumulator tile.  At
+    // d = 128 in 16-column pieces: every thread writes its row of a piece
+    // into a 64-byte-swizzled staging tile and one thread adds each 8 KB tile
+    // with a bulk reduction; with four staging tiles the first 64 columns are
+    // staged while the rest is read from TMEM.  Either way the TMEM columns
+    // are released as soon as the whole row is in registers or shared
+    // memory.  The loop is uniform over the warpgroup (named barriers are
+    // reached by every thread).
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query within the tile == TMEM lane
-    const bool leader = warp == 8 && lane == 0;
     const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + L::kColDQ;
-    const uint32_t sw = (uint32_t)(row >> 1) & 3u;  // 64-byte swizzle of this row
+    const bool leader = warp == 8 && lane == 0;
     volatile int* dq_flag = abort_flag + 1;
-    // stage 32 columns (two 16-column pieces) of this row into tiles t, t+1
+    // (d = 64) add 32 columns (8 four-column chunks from chunk c0) of this row
+    // into the chunk-major accumulator tile: chunk c of row r at
+    // (c * 128 + r) * 4 floats, so a warp's 32 rows of a chunk are 512
+    // contiguous bytes
+    auto add32 = [&](float* tile, const uint32_t (&v)[32], int c0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        red_add_v4_f32(tile + ((c0 + k) * 128 + row) * 4, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    };
+    // (d = 128) stage 32 columns (two 16-column pieces) of this row into
+    // staging tiles t, t+1 (64-byte swizzle)
+    const uint32_t sw = (uint32_t)(row >> 1) & 3u;
     auto stage = [&](const uint32_t (&v)[32], int t) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -736,63 +782,66 @@ __global__ void __launch_bounds__(448, 1)
                        v[16 * h + 4 * q4 + 2], v[16 * h + 4 * q4 + 3]);
       }
     };
-    // after a named barrier: add staging tiles 0..n-1 into pieces p0..p0+n-1
-    auto reduce = [&](float* acc_tile, int p0, int n) {
+    // (d = 128) after a named barrier: add staging tiles 0..n-1 into the
+    // tile's 16-column pieces p0..p0+n-1 (8 KB bulk reductions)
+    auto reduce = [&](float* tile, int p0, int n) {
       if (leader) {
         for (int t = 0; t < n; ++t)
-          bulk_reduce_add_f32(acc_tile + (p0 + t) * 2048, sbase + L::kOffDQ + (uint32_t)t * L::kDqPiece, L::kDqPiece);
+          bulk_reduce_add_f32(tile + (p0 + t) * 2048, sbase + L::kOffDQ + (uint32_t)t * L::kDqPiece, L::kDqPiece);
         bulk_commit();
       }
     };
     int g = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      // the leader reads the item and shares it through shared memory
-      if (leader) {
-        bool ok_ = true;
-        const int w_ = peek_item(r, ok_);
-        if (PERSIST && ok_) mbar_arrive(&bar_item_empty[r & 1]);
-        *dq_item = ok_ ? w_ : -1;
-      }
-      named_bar_sync(1, 128);
-      const int w = *reinterpret_cast<volatile int*>(dq_item);
-      named_bar_sync(1, 128);  // everyone has read it before the leader may overwrite it
-      if (w < 0) {
-        ok = false;
+      const int w = peek_item(r, ok);
+      __syncwarp();
+      if (PERSIST && ok && lane == 0) mbar_arrive(&bar_item_empty[r & 1]);
+      // the warpgroup leaves together: one flag for the whole loop
+      if (!L::kDqDirect) {
+        if (leader) *dq_flag = (ok && w < n_items) ? 1 : 0;
+        named_bar_sync(1, 128);
+        const int go = *dq_flag;
+        named_bar_sync(1, 128);
+        if (!go) break;
+      } else if (!ok || w >= n_items) {
         break;
       }
-      if (w >= n_items) break;
     const Item t = item_at(w);
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
       const int i = SPARSE ? walk.next() : q_tile(t, it);
-      // the staging tiles are free once the previous step's reductions read them
-      if (leader) {
-        bulk_wait_read<0>();
-        *dq_flag = mbar_wait(bar_dq, (g + it) & 1, ab) ? 1 : 0;
-      }
-      named_bar_sync(1, 128);
-      if (*dq_flag == 0) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float* acc_tile = a.dq_acc + ((size_t)t.bh * nT + i) * (size_t)(128 * D);
-      if (D == 64) {
+      float* tile = a.dq_acc + ((size_t)t.bh * nT + i) * (size_t)(128 * D);
+      if (L::kDqDirect) {
+        if (!mbar_wait(bar_dq, (g + it) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         uint32_t v0[32], v1[32];
         tmem_ld32(tQ, v0);
         tmem_ld32(tQ + 32u, v1);
         tmem_ld_wait();
         reg_fence(v0);
         reg_fence(v1);
+        // the whole partial is in registers: release its columns first
         tc_fence_before();
         mbar_arrive(bar_dq_free);
-        stage(v0, 0);
-        stage(v1, 2);
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        reduce(acc_tile, 0, 4);
+        add32(tile, v0, 0);
+        add32(tile, v1, 8);
       } else {
+        // the staging tiles are free once the previous step's reductions
+        // have read them; one thread waits, a named barrier shares the outcome
+        if (leader) {
+          bulk_wait_read<0>();
+          *dq_flag = mbar_wait(bar_dq, (g + it) & 1, ab) ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (*dq_flag == 0) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         {
           uint32_t v0[32], v1[32];
           tmem_ld32(tQ, v0);
@@ -813,19 +862,19 @@ __global__ void __launch_bounds__(448, 1)
         mbar_arrive(bar_dq_free);
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
-        reduce(acc_tile, 0, 4);
+        reduce(tile, 0, 4);
         if (leader) bulk_wait_read<0>();
         named_bar_sync(1, 128);
         stage(v2, 0);
         stage(v3, 2);
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
-        reduce(acc_tile, 4, 4);
+        reduce(tile, 4, 4);
       }
     }
     g += t.n_steps;
     }
-    if (leader) bulk_wait_all();
+    if (!L::kDqDirect && leader) bulk_wait_all();
   } else if (run && warp < 8) {
     // --------------------------------------------------------- P and dS
     const int wg = warp >> 2;
