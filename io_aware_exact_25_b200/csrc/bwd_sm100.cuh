@@ -42,6 +42,7 @@
 //   warps 8-11  dQ read-out and accumulation               (TMEM lanes = queries)
 //   warp  12    tcgen05 MMA issue (one thread)
 //   warp  13    TMA producer (+ dropout row keys)
+//   warps 14-15 idle (they complete warpgroup 3 for the register split)
 // Tensor memory (512 columns): R_S [0,128) S^T fp32, then P^T bf16 in
 // [0,32) and [64,96); R_dP [128,256) dP^T fp32, then (d = 128) the dQ
 // partial (fp32, D columns); dV at 256, dK at 256 + D; at d = 64 the dQ
@@ -270,7 +271,16 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
 
 template <int D, bool DROPOUT>
 struct BwdLayout {
-  static constexpr int kThreads = 448;
+  // 16 warps: P/dS warpgroups 0-1, dQ warpgroup 2, and warpgroup 3 (MMA
+  // issue, TMA producer, two idle warps) so that every warpgroup is whole for
+  // the register reallocation: launched at 128 registers a thread (the whole
+  // register file), then 160 for the P/dS warpgroups, 104 for dQ and 80 for
+  // warpgroup 3 -- 2*4*32*160 + 4*32*104 + 4*32*80 = 64512 <= 65536.  (At 128
+  // registers for every warp the dropout kernels spilled 220-280 bytes a
+  // thread; with this split 12.)
+  static constexpr int kThreads = 512;
+  static constexpr uint32_t kRegsPS = 160, kRegsDQ = 104, kRegsCtl = 80;
+  static_assert(2 * 128 * kRegsPS + 128 * kRegsDQ + 128 * kRegsCtl <= 512 * 128, "register split");
   static constexpr uint32_t kHalf = 128u * 128u;
   static constexpr uint32_t kTile = 128u * D * 2u;
   static constexpr int kQStages = 2;
@@ -323,11 +333,13 @@ __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8u * kk
 constexpr bool kRotateQueryTiles = false;
 
 // Of every 8 pairs of recomputed probabilities, this many take the
-// exponential on the FMA pipe (polynomial), the rest on MUFU.
-constexpr int kBwdPolyPairsOf8 = 0;
+// exponential on the FMA pipe (polynomial), the rest on MUFU.  Measured: 2 of
+// 8 is 1.4% faster at d = 128 (3.6% with dropout) and 2-4% slower at d = 64.
+template <int D>
+__host__ __device__ constexpr int bwd_poly_pairs_of8() { return D == 128 ? 2 : 0; }
 
 template <int D, bool CAUSAL, bool DROPOUT, bool SPARSE, bool VARLEN>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const BwdArgs a) {
@@ -502,6 +514,10 @@ __global__ void __launch_bounds__(448, 1)
     return t;
   };
 
+  // Each warpgroup sets its register budget at the top of its branch (every
+  // thread of the warpgroup, whatever its role or the abort state).
+  if (warp >= 12) {
+  regs_dec<L::kRegsCtl>();
   if (run && warp == 13) {
     // ------------------------------------------------------ TMA producer
     const uint64_t pol_keep = policy_evict_last();
@@ -742,7 +758,10 @@ __global__ void __launch_bounds__(448, 1)
         mbar_wait_drain(bar_drain, 0);
       }
     }
-  } else if (run && warp >= 8 && warp < 12) {
+  }
+  } else if (warp >= 8) {
+  regs_dec<L::kRegsDQ>();
+  if (run) {
     // ------------------------------------------ dQ read-out + accumulate
     // The partial dQ_i (128 rows x D fp32, query rows on the TMEM lanes) is
     // added into the fp32 accumulator.  At d = 64 straight from registers
@@ -875,7 +894,10 @@ __global__ void __launch_bounds__(448, 1)
     g += t.n_steps;
     }
     if (!L::kDqDirect && leader) bulk_wait_all();
-  } else if (run && warp < 8) {
+  }
+  } else {
+  regs_inc<L::kRegsPS>();
+  if (run) {
     // --------------------------------------------------------- P and dS
     const int wg = warp >> 2;
     const int quad = warp & 3;
@@ -918,8 +940,8 @@ __global__ void __launch_bounds__(448, 1)
       reg_fence(u[1]);
       // P^T_jq = 2^(s * scale * log2 e - lse2_q); padded queries have lse2 = +inf.
       // Scale/subtract on the packed f32x2 pipe; of every 8 pairs,
-      // kBwdPolyPairsOf8 take the exponential on the FMA pipe (polynomial),
-      // the rest on MUFU.
+      // bwd_poly_pairs_of8 take the exponential on the FMA pipe
+      // (polynomial), the rest on MUFU.
       float p[64];
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
@@ -930,7 +952,7 @@ __global__ void __launch_bounds__(448, 1)
           const int c = 4 * c4 + 2 * e2;
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[c >> 5][c & 31]), __uint_as_float(u[c >> 5][(c + 1) & 31])),
                                      sl2x2, f2_pack(e2 ? -l4.z : -l4.x, e2 ? -l4.w : -l4.y));
-          if (((c >> 1) & 7) < kBwdPolyPairsOf8) {
+          if (((c >> 1) & 7) < bwd_poly_pairs_of8<D>()) {
             exp2_poly_x2(x2, p[c], p[c + 1]);
           } else {
             float x0, x1;
@@ -1087,6 +1109,7 @@ __global__ void __launch_bounds__(448, 1)
     }
     g += t.n_steps;
     }
+  }
   }
 
   tc_fence_before();
