@@ -171,6 +171,21 @@ def oracle_step(x, w, n_rows: int, mask=None):
     return dt, 3.5 * f
 
 
+def varlen_oracle_step(x, w, n_rows: int):
+    """fp64 oracle forward + full backward of head 0 of the first sequence of
+    a packed variable-length batch, its first n_rows tokens (an exact
+    sub-problem under the causal mask).  Returns (seconds, FLOPs)."""
+    import oracle
+    L0 = min(w.lens[0], n_rows)
+    q, k, v, do = (x[n][:L0, :1].transpose(0, 1).unsqueeze(0).contiguous() for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    oracle.backward_q(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    oracle.backward_kv(q, k, v, do, w.scale, causal=w.causal, p_drop=w.p_drop, seed=w.seed)
+    dt = time.perf_counter() - t0
+    return dt, 3.5 * 4.0 * L0 * L0 * w.d * (0.5 if w.causal else 1.0)
+
+
 def oracle_full(x, w):
     """fp64 oracle forward + full backward on every head and row of the
     workload.  Returns (seconds, FLOPs by the attention convention)."""
@@ -190,9 +205,12 @@ def run_reference(args, w):
     from io_aware_exact_25_b200.inputs import workload_inputs
     import oracle
     x = workload_inputs(w)
-    n_rows = min(args.ref_rows, w.N)
-    full = args.ref_full
-    step = (lambda: oracle_full(x, w)) if full else (lambda: oracle_step(x, w, n_rows))
+    n_rows = min(args.ref_rows, w.lens[0] if w.lens else w.N)
+    full = args.ref_full and not w.lens
+    if w.lens:
+        step = lambda: varlen_oracle_step(x, w, n_rows)
+    else:
+        step = (lambda: oracle_full(x, w)) if full else (lambda: oracle_step(x, w, n_rows))
     for _ in range(args.warmup):
         step()
     tot_t, tot_f = 0.0, 0.0
@@ -202,7 +220,8 @@ def run_reference(args, w):
         tot_f += f
     value = tot_f / tot_t / 1e12
     sample = (f"per step: fwd+bwd of the whole workload ({w.B * w.H} heads x {w.N} rows)" if full else
-              f"per step: fwd+bwd of the {'causal ' if w.causal else ''}prefix N={n_rows} of head (0,0)")
+              f"per step: fwd+bwd of the {'causal ' if w.causal else ''}prefix N={n_rows} of head (0,0)"
+              + (" (sequence 0 of the packed batch)" if w.lens else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -216,12 +235,23 @@ def run_reference(args, w):
     if not full:
         # the prefix is an exact sub-problem whose work grows as n^2; the whole
         # workload is B*H heads of length N
-        line["extrapolated_full_problem_s"] = (tot_t / args.steps) * w.B * w.H * (w.N / n_rows) ** 2
+        lens = w.lens or (w.N,) * w.B
+        line["extrapolated_full_problem_s"] = (tot_t / args.steps) * w.H * sum((L / n_rows) ** 2 for L in lens)
     print(json.dumps(line), flush=True)
     return 0
 
 
 def workload_config(w, mask_kind=None, frac=None):
+    if w.lens:
+        T = sum(w.lens)
+        tensor_mib = T * w.H * w.d * 2 / 2 ** 20
+        return {"workload": f"{w.name}: {w.B} sequences of {min(w.lens)}-{max(w.lens)} tokens (total {T}) packed "
+                            f"token-major, H={w.H} d={w.d} {'causal' if w.causal else 'non-causal'} "
+                            f"dropout={w.p_drop} bf16",
+                "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "dropout_p": w.p_drop,
+                "lens": list(w.lens), "total_tokens": T,
+                "l2": f"inputs larger than L2 (Q, K, V, dO: 4 x {tensor_mib:.0f} MiB per step > 126 MB L2)",
+                "parallelism": "replicas: each GPU runs its own batch, no collective"}
     tensor_mib = w.B * w.H * w.N * w.d * 2 / 2 ** 20
     cfg = {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
                        f"{'causal' if w.causal else 'non-causal'} dropout={w.p_drop} bf16",
@@ -540,6 +570,175 @@ def run_ours(args, w):
     return 0
 
 
+def run_ours_varlen(args, w):
+    """One step = fa_fwd_varlen + fa_bwd_varlen over a packed variable-length
+    batch; FLOPs summed over the sequences (Workload.fwd_flops)."""
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    from io_aware_exact_25_b200 import binding
+    from io_aware_exact_25_b200.inputs import workload_inputs
+    lib = binding.load()
+    x = workload_inputs(w)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    cu = x["cu_seqlens"].to(dev)
+    T, H, d = q.shape
+    B, maxs = w.B, w.N
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = int(lib.fa_bwd_varlen_workspace_size(B, H, maxs, d))
+    work = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev).cuda_stream
+    P = binding._ptr
+    S4 = binding._tok_strides(q, k, v, o)
+    S8 = binding._tok_strides(q, k, v, o, do, dq, dk, dv)
+    causal = int(w.causal)
+
+    def check(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: {binding.strerror(rc)}")
+
+    def fwd():
+        check(lib.fa_fwd_varlen(P(q), P(k), P(v), P(o), P(lse), S4, P(cu), None, B, H, maxs, T, d, w.scale, causal,
+                                w.p_drop, w.seed, s), "fa_fwd_varlen")
+
+    def bwd():
+        check(lib.fa_bwd_varlen(P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), S8, P(cu), None, B, H,
+                                maxs, T, d, w.scale, causal, w.p_drop, w.seed, P(work), wsb, s), "fa_bwd_varlen")
+
+    # fa_bwd_varlen launches bwd_pre_kernel, bwd_kernel and bwd_post_kernel
+    stages = [("fwd_kernel", fwd), ("bwd_pre_kernel + bwd_kernel + bwd_post_kernel", bwd)]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        for _, fn in stages:
+            fn()
+    torch.cuda.synchronize(dev)
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error during warm-up")
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for st in range(args.steps):
+        ev[st][0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            ev[st][i + 1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    stage_ms = [sum(ev[st][i].elapsed_time(ev[st][i + 1]) for st in range(args.steps)) / args.steps
+                for i in range(len(stages))]
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error in the timed region")
+    ok = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all()
+              and torch.isfinite(dv.float()).all())
+    # per sequence and head: sum_j dK_j = 0 and, without dropout, sum_j dV_j = sum_i dO_i
+    seg = torch.repeat_interleave(torch.arange(B, device=dev), torch.tensor(w.lens, device=dev))
+
+    def seg_sum(t):
+        return torch.zeros((B, H, d), dtype=torch.float32, device=dev).index_add_(0, seg, t.float())
+
+    ok = ok and bool((seg_sum(dk).abs() <= 1e-2 * seg_sum(dk.abs()) + 1e-2).all())
+    if w.p_drop == 0.0:
+        ok = ok and bool(((seg_sum(dv) - seg_sum(do)).abs() <= 1e-2 * seg_sum(dv.abs()) + 1e-2).all())
+    # end to end through the public API: pinned host inputs in, results out
+    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
+    h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (o, lse, dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
+            dst.copy_(src, non_blocking=True)
+        binding.fwd_varlen(q, k, v, cu, maxs, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
+                           o=o, lse=lse)
+        binding.bwd_varlen(q, k, v, o, do, lse, cu, maxs, causal=w.causal, scale=w.scale, dropout_p=w.p_drop,
+                           seed=w.seed, dq=dq, dk=dk, dv=dv, workspace=work)
+        for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    from io_aware_exact_25_b200.replicas import replica_summary
+    summ = replica_summary(elapsed_ms, e2e_ms, stage_ms, ok, device=dev)
+    if not summ["all_ok"]:
+        raise RuntimeError("a replica's outputs failed their checks")
+    if rank == 0:
+        ff, fb = w.fwd_flops(), w.bwd_flops()
+        ms_step = summ["elapsed_ms"] / args.steps
+        value = ws * (ff + fb) / (ms_step * 1e-3) / 1e12
+        peaks, peak_kind = load_peaks()
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        long_region = summ["elapsed_ms"] >= LONG_REGION_MS
+        roof_peak = sustained if long_region else burst
+        fwd_ms, bwd_ms = summ["stage_ms"]
+        dom = 0 if fwd_ms > bwd_ms else 1
+        dom_flops = ff if dom == 0 else fb
+        achieved = dom_flops / ((fwd_ms if dom == 0 else bwd_ms) * 1e-3) / 1e12
+        # the CPU baseline: the oracle on the first sequence of the batch, head 0
+        import oracle
+        L0 = min(w.lens[0], args.cpu_rows)
+        cpu_dt, cpu_f = varlen_oracle_step(x, w, L0)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "fwd_tflops": ws * ff / (fwd_ms * 1e-3) / 1e12, "fwd_bwd_tflops": value,
+            "frac_of_peak": {"fwd_vs_burst": (ff / (fwd_ms * 1e-3) / 1e12) / burst,
+                             "fwd_bwd_vs_burst": (value / ws) / burst,
+                             "fwd_bwd_vs_datasheet": (value / ws) / DATASHEET_BF16_TFLOPS,
+                             "peaks": f"{peak_kind}: burst {burst}, sustained {sustained}"},
+            "stage_ms": dict(zip([n for n, _ in stages], summ["stage_ms"])),
+            "roofline": {"bound": "tensor", "kernel": stages[dom][0], "achieved": achieved, "peak": roof_peak,
+                         "unit": "TFLOP/s", "frac": achieved / roof_peak,
+                         "peak_note": f"{'bf16_tflops_sustained' if long_region else 'bf16_tflops (burst)'} of "
+                                      f"{peak_kind}: the timed region is {summ['elapsed_ms']:.1f} ms",
+                         "traffic": None, "algorithmic_flops_per_launch": dom_flops},
+            "cpu_baseline": {"value": cpu_f / cpu_dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"fp64 fwd+bwd of sequence 0 (first {L0} tokens), head 0 ({cpu_dt:.1f} s)"},
+            "e2e": {"value": ws * (ff + fb) * e2e_steps / (summ["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "binding.fwd_varlen/binding.bwd_varlen (C ABI) with pinned host buffers, one stream"},
+            "gpu_launches": args.steps * (1 + 3),
+            "replica_checks": {"ranks": ws, "all_ok": summ["all_ok"],
+                               "checks": "finite outputs; per sequence and head sum_j dK_j = 0 and "
+                                         "sum_j dV_j = sum_i dO_i"},
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -571,6 +770,8 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if w.lens:
+        return run_ours_varlen(args, w)
     return run_ours(args, w)
 
 

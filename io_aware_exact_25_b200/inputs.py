@@ -38,20 +38,36 @@ class Workload:
     seed: int
     qkv_scale: float = 1.0
     offset_norm: float = 0.0
+    # variable-length batch: the B sequence lengths (N is the longest); empty
+    # for a dense [B, H, N, d] workload
+    lens: tuple = ()
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def fwd_flops(self) -> float:
-        """4*B*H*N^2*d, halved when causal (the attention FLOP convention)."""
-        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        """4*B*H*N^2*d, halved when causal (the attention FLOP convention);
+        a variable-length batch sums 4*H*L^2*d over its sequences."""
+        if self.lens:
+            f = sum(4.0 * self.H * L * L * self.d for L in self.lens)
+        else:
+            f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2.0 if self.causal else f
 
     def bwd_flops(self) -> float:
         """2.5x the forward (five GEMMs against two)."""
         return 2.5 * self.fwd_flops()
 
+
+def varlen_lengths(count: int, lo: int, hi: int, seed: int) -> tuple:
+    """``count`` sequence lengths drawn uniformly from [lo, hi] by a torch
+    generator seeded with ``2000 + seed`` (a mixed-length training batch)."""
+    g = torch.Generator().manual_seed(2000 + int(seed))
+    return tuple(int(x) for x in torch.randint(lo, hi + 1, (count,), generator=g))
+
+
+_MIX = varlen_lengths(16, 512, 8192, 6)
 
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, 128, 64, False, 0.0, 0),
@@ -62,6 +78,9 @@ WORKLOADS = {
     "long64k_causal_dropout": Workload("long64k_causal_dropout", 1, 8, 65536, 128, True, 0.1, 4),
     # few query tiles (64 CTAs of work for 148 SMs): the split-KV case
     "smallbatch16k": Workload("smallbatch16k", 1, 1, 16384, 128, False, 0.0, 5),
+    # a variable-length batch: 16 sequences of 512-8192 tokens packed back to
+    # back (token-major), causal, d = 128
+    "varlen_mix": Workload("varlen_mix", len(_MIX), 16, max(_MIX), 128, True, 0.0, 6, lens=_MIX),
 }
 
 
@@ -88,6 +107,20 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int, qkv_scale: float = 1.
 
 
 def workload_inputs(w: Workload) -> dict:
+    """Dense workloads: ``{'q','k','v','do'}`` bf16 ``[B,H,N,d]``.  Variable-length
+    workloads: the same keys as token-major bf16 ``[T, H, d]`` (T = sum of the
+    lengths, drawn in the order Q, K, V, dO as fp32 randn of that shape) plus
+    ``'cu_seqlens'``, int32 ``[B+1]`` offsets."""
+    if w.lens:
+        g = torch.Generator().manual_seed(int(w.seed))
+        T = sum(w.lens)
+        out = {n: torch.randn((T, w.H, w.d), generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+               for n in ("q", "k", "v", "do")}
+        cu = [0]
+        for L in w.lens:
+            cu.append(cu[-1] + L)
+        out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
+        return out
     return make_inputs(w.B, w.H, w.N, w.d, w.seed, w.qkv_scale, w.offset_norm)
 
 
