@@ -340,6 +340,17 @@ int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const i
 int fa_debug_fwd_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
                          int d, float scale, int causal, void* stream);
 
+/*
+ * Test hook for the polynomial exponential (the paper has no counterpart):
+ * y[i] = 2^x[i] computed by the device function the backward kernel uses for
+ * part of its recomputed probabilities (a Cody-Waite split and a cubic
+ * minimax fit on the FMA pipe), so that tests can hold it to its stated
+ * error bound against CUDA's exp2.  x and y are device pointers to n floats
+ * (n >= 0; 4-byte aligned).  Returns FA_ERR_INVALID_ARG for n < 0 or null
+ * pointers with n > 0; asynchronous on `stream`.
+ */
+int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
+
 /* Static description of a status code. */
 const char* fa_strerror(int status);
 

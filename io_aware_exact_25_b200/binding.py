@@ -30,7 +30,7 @@ FA_ERR_TOO_LARGE = -7
 EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
-           "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout",
+           "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout", "fa_debug_exp2_poly",
            "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
            "fa_fwd_partial", "fa_merge_partials", "fa_bwd_dq_accumulator_bytes", "fa_bwd_recompute_range",
            "fa_dropout_mask", "fa_strerror",
@@ -81,6 +81,7 @@ def load() -> ctypes.CDLL:
         lib.fa_bwd_recompute_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, I, vp, SZ,
                                                      vp]
         lib.fa_debug_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, vp]
+        lib.fa_debug_exp2_poly.argtypes = [vp, vp, I, vp]
         lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         lib.fa_bwd_workspace_size.restype = SZ
         lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
@@ -104,7 +105,7 @@ def load() -> ctypes.CDLL:
         for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
                    lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
                    lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
-                   lib.fa_debug_fwd_timeout, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
+                   lib.fa_debug_fwd_timeout, lib.fa_debug_exp2_poly, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
                    lib.fa_merge_partials, lib.fa_bwd_recompute_range,
                    lib.fa_dropout_mask, lib.fa_get_device_error,
                    lib.fa_last_cuda_error, lib.fa_version):
@@ -498,6 +499,16 @@ def debug_fwd_timeout(q, k, v, causal=False, scale=None, stream=None) -> int:
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     return int(load().fa_debug_fwd_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
                                            int(bool(causal)), _stream(stream)))
+
+
+def debug_exp2_poly(x, stream=None):
+    """2^x through the kernels' polynomial exponential (``fa_debug_exp2_poly``),
+    for tests; x is a float32 CUDA tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _call(load().fa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "fa_debug_exp2_poly")
+    return y
 
 
 def device_error(stream=None) -> int:

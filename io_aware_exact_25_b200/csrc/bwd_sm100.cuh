@@ -25,7 +25,8 @@
 //     accumulates dV += P^T dO_i (P^T from tensor memory) and dK += dS^T Q_i
 //     (dS from shared memory) in tensor memory, and
 //     computes the dQ_i partial dS K_j, which a warpgroup adds into the fp32
-//     accumulator from registers with vector reductions;
+//     accumulator (d = 64: from registers with vector reductions; d = 128:
+//     staged in shared memory, one 8 KB bulk reduction per piece);
 //  3. dQ = scale * accumulator, rounded to bf16.
 // Variable-length mode ("FlashAttention for Efficient Training" section 5.2):
 // sequences stored token-major at offsets cu_seqlens; a CTA's item is a key

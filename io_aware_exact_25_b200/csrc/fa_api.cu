@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -380,6 +381,29 @@ int fa_debug_fwd_timeout(const void* q, const void* k, const void* v, void* o, f
   const fa_strides s = contiguous_strides(H, N, d);
   const fa_strides all[4] = {s, s, s, s};
   return fwd_impl(q, k, v, o, lse, all, B, H, N, d, scale, causal, 0.f, 0, 1, nullptr, 0, nullptr, 0, stream, 1);
+}
+
+namespace {
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int stride = 2 * gridDim.x * blockDim.x;
+  for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += stride) {
+    const bool two = i + 1 < n;
+    float r0, r1;
+    fa::exp2_poly_x2(fa::f2_pack(x[i], two ? x[i + 1] : 0.f), r0, r1);
+    y[i] = r0;
+    if (two) y[i + 1] = r1;
+  }
+}
+}  // namespace
+
+int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!aligned(x, 4) || !aligned(y, 4)) return FA_ERR_ALIGNMENT;
+  const int blocks = (int)std::min<long long>(148 * 8, ((long long)n + 511) / 512);
+  exp2_poly_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 int fa_dropout_mask(int B, int H, int N, float dropout_p, uint64_t seed, const int32_t* heads, int nheads,

@@ -404,7 +404,8 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 }
 
 // 2^x for two values at once on the FMA pipe, for x <= 126 (x = -inf or
-// below -126 gives a value below 2^-125 instead of 0).  Cody-Waite split
+// below -125 gives a value in [0, 2^-124] instead of 2^x: the
+// exponent arithmetic leaves the normal range).  Cody-Waite split
 // x = n + f with n = round(x) and f in [-1/2, 1/2]: n comes from adding
 // 1.5 * 2^23 (the rounded integer lands in the low mantissa bits), 2^f from a
 // cubic, and n is added to the exponent field with integer arithmetic.  The

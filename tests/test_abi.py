@@ -136,6 +136,12 @@ def test_empty_problems_are_noops(lib):
     assert _fwd(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == binding.FA_OK
     assert _bwd(lib, ptr=None, lse=None, H=0, ws=None, wsb=0) == binding.FA_OK
     assert lib.fa_dropout_mask(1, 1, 0, 0.1, 0, None, 0, None, 0, None, None) == binding.FA_OK
+    assert lib.fa_debug_exp2_poly(None, None, 0, None) == binding.FA_OK
+
+
+def test_exp2_hook_rejects_bad_arguments(lib):
+    assert lib.fa_debug_exp2_poly(None, None, -1, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_debug_exp2_poly(None, None, 4, None) == binding.FA_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("B,H,N,d", [(1, 2, 128, 64), (2, 16, 8192, 128), (1, 3, 300, 128), (1, 1, 1, 64)])
