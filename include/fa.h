@@ -351,6 +351,26 @@ int fa_debug_fwd_timeout(const void* q, const void* k, const void* v, void* o, f
  */
 int fa_debug_exp2_poly(const float* x, float* y, int n, void* stream);
 
+/*
+ * The bounds-checking build (the paper has no counterpart).  The library
+ * also builds as libfa_sm100_debug.so, compiled with FA_DEBUG: there every
+ * global-memory access the kernels derive from their work decomposition
+ * (output rows, dQ accumulator tiles, row statistics, split-KV pieces, work
+ * items, TMA tile rows) is checked against the extent its buffer has by the
+ * call's shape and strides before it is made.  A failed check skips the
+ * access (a tile load is still issued: out-of-range rows read as zero),
+ * sets device error 4 and records the first failure.
+ *
+ * fa_debug_build returns 1 in that build and 0 in the release build.
+ * fa_debug_bounds_record synchronises `stream`, copies the record into
+ * out[0..5] = {failed checks, site, offset, limit, block, thread} (offsets in
+ * elements; site numbers are listed in csrc/debug_check.cuh) and clears it;
+ * the release build returns FA_ERR_UNSUPPORTED.  out is a host pointer to 6
+ * long longs.
+ */
+int fa_debug_build(void);
+int fa_debug_bounds_record(long long* out, void* stream);
+
 /* Static description of a status code. */
 const char* fa_strerror(int status);
 
@@ -361,7 +381,8 @@ int fa_last_cuda_error(void);
  * Synchronises `stream`, then reads and clears the calling device's error
  * word.  Returns 0 if no kernel reported an error since the last read, else
  * the kernel's code (1 = a bounded wait timed out, 2 = shared memory
- * misaligned, 3 = variable-length offsets or lengths out of range);
+ * misaligned, 3 = variable-length offsets or lengths out of range, 4 = a
+ * bounds check failed, bounds-checking build only);
  * FA_ERR_CUDA if the synchronisation itself failed.
  */
 int fa_get_device_error(void* stream);

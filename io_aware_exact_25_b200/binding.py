@@ -8,6 +8,7 @@ library or a non-CUDA tensor raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -17,6 +18,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libfa_sm100_debug.so")  # the bounds-checking build (FA_DEBUG)
 
 FA_OK = 0
 FA_ERR_INVALID_ARG = -1
@@ -31,6 +33,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspa
            "fa_splitkv_suggest", "fa_bwd", "fa_bwd_strided", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_recompute",
            "fa_bwd_finalize", "fa_bwd_noalloc", "fa_fwd_blocksparse", "fa_bwd_blocksparse",
            "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout", "fa_debug_exp2_poly",
+           "fa_debug_build", "fa_debug_bounds_record",
            "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
            "fa_fwd_partial", "fa_merge_partials", "fa_bwd_dq_accumulator_bytes", "fa_bwd_recompute_range",
            "fa_dropout_mask", "fa_strerror",
@@ -54,64 +57,94 @@ class FaError(RuntimeError):
 
 
 def load() -> ctypes.CDLL:
-    """Load ``libfa_sm100.so`` (raises if it has not been built)."""
+    """Load ``libfa_sm100.so`` (raises if it has not been built); every
+    function of this module calls through it."""
     global _lib
     with _lock:
         if _lib is not None:
             return _lib
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; build it with "
-                               "io_aware_exact_25_b200.build.build()")
-        lib = ctypes.CDLL(LIB_PATH)
-        vp, I, F, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
-        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
-        lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, vp, SZ, vp]
-        lib.fa_fwd_splitkv_workspace_size.argtypes = [I, I, I, I, I]
-        lib.fa_fwd_splitkv_workspace_size.restype = SZ
-        lib.fa_splitkv_suggest.argtypes = [I, I, I, I]
-        lib.fa_splitkv_suggest.restype = I
-        SP = ctypes.POINTER(FaStrides)
-        lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp]
-        lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, SZ,
-                                       vp]
-        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
-        lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I, vp]
-        lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I,
-                                           vp, SZ, vp]
-        lib.fa_bwd_recompute_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, I, vp, SZ,
-                                                     vp]
-        lib.fa_debug_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, vp]
-        lib.fa_debug_exp2_poly.argtypes = [vp, vp, I, vp]
-        lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
-        lib.fa_bwd_workspace_size.restype = SZ
-        lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
-        lib.fa_bwd_recompute.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
-        lib.fa_bwd_finalize.argtypes = [vp, I, I, I, I, F, vp, SZ, vp]
-        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
-        lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
-        lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64, vp]
-        lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64,
-                                      vp, SZ, vp]
-        lib.fa_bwd_varlen_workspace_size.argtypes = [I, I, I, I]
-        lib.fa_bwd_varlen_workspace_size.restype = SZ
-        lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp]
-        lib.fa_merge_partials.argtypes = [vp, vp, I, vp, vp, I, I, I, I, vp]
-        lib.fa_bwd_dq_accumulator_bytes.argtypes = [I, I, I, I]
-        lib.fa_bwd_dq_accumulator_bytes.restype = SZ
-        lib.fa_bwd_recompute_range.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp, SZ, vp]
-        lib.fa_strerror.argtypes = [I]
-        lib.fa_strerror.restype = ctypes.c_char_p
-        lib.fa_get_device_error.argtypes = [vp]
-        for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
-                   lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
-                   lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
-                   lib.fa_debug_fwd_timeout, lib.fa_debug_exp2_poly, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
-                   lib.fa_merge_partials, lib.fa_bwd_recompute_range,
-                   lib.fa_dropout_mask, lib.fa_get_device_error,
-                   lib.fa_last_cuda_error, lib.fa_version):
-            fn.restype = I
+        _lib = _open(LIB_PATH)
+        return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route every call of this module through another build of the library
+    (``DEBUG_LIB_PATH``, the bounds-checking build) inside the block."""
+    global _lib
+    lib = _open(path)
+    with _lock:
+        saved = _lib
         _lib = lib
-        return lib
+    try:
+        yield lib
+    finally:
+        with _lock:
+            _lib = saved
+
+
+def debug_bounds_record(stream=None) -> list:
+    """The bounds-checking build's record of its first failed check
+    ({failed checks, site, offset, limit, block, thread}), cleared by reading."""
+    out = (ctypes.c_longlong * 6)()
+    _call(load().fa_debug_bounds_record(out, _stream(stream)), "fa_debug_bounds_record")
+    return list(out)
+
+
+def _open(path: str) -> ctypes.CDLL:
+    """Open one build of the library and declare its signatures."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing; build it with io_aware_exact_25_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    vp, I, F, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, vp, SZ, vp]
+    lib.fa_fwd_splitkv_workspace_size.argtypes = [I, I, I, I, I]
+    lib.fa_fwd_splitkv_workspace_size.restype = SZ
+    lib.fa_splitkv_suggest.argtypes = [I, I, I, I]
+    lib.fa_splitkv_suggest.restype = I
+    SP = ctypes.POINTER(FaStrides)
+    lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp]
+    lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, SZ,
+                                   vp]
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
+    lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I, vp]
+    lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, I, I, I, I, F, I, F, U64, vp, I,
+                                       vp, SZ, vp]
+    lib.fa_bwd_recompute_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, I, vp, SZ,
+                                                 vp]
+    lib.fa_debug_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, vp]
+    lib.fa_debug_exp2_poly.argtypes = [vp, vp, I, vp]
+    lib.fa_debug_bounds_record.argtypes = [vp, vp]
+    lib.fa_bwd_workspace_size.argtypes = [I, I, I, I]
+    lib.fa_bwd_workspace_size.restype = SZ
+    lib.fa_bwd_prepare.argtypes = [vp, vp, vp, I, I, I, I, vp, SZ, vp]
+    lib.fa_bwd_recompute.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp, SZ, vp]
+    lib.fa_bwd_finalize.argtypes = [vp, I, I, I, I, F, vp, SZ, vp]
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, vp]
+    lib.fa_dropout_mask.argtypes = [I, I, I, F, U64, vp, I, vp, I, vp, vp]
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64, vp]
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, SP, vp, vp, I, I, I, I, I, F, I, F, U64,
+                                  vp, SZ, vp]
+    lib.fa_bwd_varlen_workspace_size.argtypes = [I, I, I, I]
+    lib.fa_bwd_varlen_workspace_size.restype = SZ
+    lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp]
+    lib.fa_merge_partials.argtypes = [vp, vp, I, vp, vp, I, I, I, I, vp]
+    lib.fa_bwd_dq_accumulator_bytes.argtypes = [I, I, I, I]
+    lib.fa_bwd_dq_accumulator_bytes.restype = SZ
+    lib.fa_bwd_recompute_range.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp, SZ, vp]
+    lib.fa_strerror.argtypes = [I]
+    lib.fa_strerror.restype = ctypes.c_char_p
+    lib.fa_get_device_error.argtypes = [vp]
+    for fn in (lib.fa_fwd, lib.fa_fwd_splitkv, lib.fa_fwd_strided, lib.fa_bwd_strided, lib.fa_bwd,
+               lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
+               lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
+               lib.fa_debug_fwd_timeout, lib.fa_debug_exp2_poly, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
+               lib.fa_merge_partials, lib.fa_bwd_recompute_range,
+               lib.fa_dropout_mask, lib.fa_get_device_error,
+               lib.fa_last_cuda_error, lib.fa_version, lib.fa_debug_build, lib.fa_debug_bounds_record):
+        fn.restype = I
+    return lib
 
 
 def strerror(status: int) -> str:

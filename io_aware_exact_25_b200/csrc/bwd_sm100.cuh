@@ -53,6 +53,7 @@
 // of one step overlaps dK and the next step's P.
 #pragma once
 
+#include "debug_check.cuh"
 #include "dropout_hash.cuh"
 #include "sm100.cuh"
 
@@ -138,6 +139,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
   constexpr int kRpw = 32 / kTpr;   // rows per warp per group
   constexpr int kU = 4;             // groups in flight
   const long long rows = (long long)BH * npad;
+  // buffer extents for the bounds-checking build (unused otherwise)
+  const bool vl = a.cu_seqlens != nullptr;
+  const long long rows_t = vl ? a.total_tokens : a.N;
+  const long long o_lim = extent4(vl ? 1 : a.B, a.H, rows_t, D, a.o_sb, a.o_sh, a.o_sn);
+  const long long do_lim = extent4(vl ? 1 : a.B, a.H, rows_t, D, a.do_sb, a.do_sh, a.do_sn);
+  const long long lse_lim = vl ? (long long)a.H * a.total_tokens : (long long)BH * a.N;
+  (void)o_lim, (void)do_lim, (void)lse_lim;
   const int lane = threadIdx.x & 31;
   const int sub = lane / kTpr, part = lane - sub * kTpr;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
@@ -161,8 +169,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
         }
         if (i < len) {
           const long long row = row0 + i;
-          ov[u] = *reinterpret_cast<const uint4*>(a.o + b_ * a.o_sb + h_ * a.o_sh + row * a.o_sn + 8 * part);
-          dv[u] = *reinterpret_cast<const uint4*>(a.dout + b_ * a.do_sb + h_ * a.do_sh + row * a.do_sn + 8 * part);
+          const long long ooff = b_ * a.o_sb + h_ * a.o_sh + row * a.o_sn + 8 * part;
+          const long long doff = b_ * a.do_sb + h_ * a.do_sh + row * a.do_sn + 8 * part;
+          if (FA_IN(kSiteBwdPreRow, ooff, 8, o_lim, a.err) && FA_IN(kSiteBwdPreRow, doff, 8, do_lim, a.err)) {
+            ov[u] = *reinterpret_cast<const uint4*>(a.o + ooff);
+            dv[u] = *reinterpret_cast<const uint4*>(a.dout + doff);
+          }
         }
       }
     }
@@ -188,7 +200,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a, int BH, i
           lse_at = (long long)h_ * a.total_tokens + sp.row0 + i;
         }
         a.drow[r] = i < len ? acc : 0.f;
-        a.lse2[r] = i < len ? a.lse[lse_at] * 1.4426950408889634f : INFINITY;
+        const bool l_ok = i >= len || FA_IN(kSiteBwdPreLse, lse_at, 1, lse_lim, a.err);
+        a.lse2[r] = i < len && l_ok ? a.lse[lse_at] * 1.4426950408889634f : INFINITY;
       }
     }
   }
@@ -211,11 +224,15 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                        int BH, int H, int N, long long sb, long long sh, long long sn,
                                                        float scale, const int* cu_seqlens, const int* seqused,
-                                                       int total_tokens) {
+                                                       int total_tokens, int* err) {
   constexpr bool kChunkMajor = D == 64;
   const int nT = (N + 127) >> 7;
   constexpr int kC8 = D / 8;  // chunk pairs per row
   const long long n = (long long)BH * nT * 128 * kC8;
+  // buffer extents for the bounds-checking build (unused otherwise)
+  const long long acc_lim = (long long)BH * nT * 128 * D;
+  const long long dq_lim = extent4(cu_seqlens ? 1 : BH / H, H, cu_seqlens ? total_tokens : N, D, sb, sh, sn);
+  (void)acc_lim, (void)dq_lim, (void)err;
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n;
        u += (long long)gridDim.x * blockDim.x) {
     int c8, r, tile, bh;
@@ -246,7 +263,10 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
       row = sp.row0 + i;
     }
     if (i >= len) continue;
-    const float* blk = acc + ((size_t)bh * nT + tile) * (size_t)(128 * D);
+    const long long blk_off = ((long long)bh * nT + tile) * (128 * D);
+    const long long dq_off = b_ * sb + h_ * sh + row * sn + 8 * c8;
+    if (!FA_IN(kSiteBwdPost, blk_off, 128 * D, acc_lim, err) || !FA_IN(kSiteBwdPost, dq_off, 8, dq_lim, err)) continue;
+    const float* blk = acc + blk_off;
     float4 x, y;
     if (kChunkMajor) {
       x = *reinterpret_cast<const float4*>(blk + ((2 * c8) * 128 + r) * 4);
@@ -264,7 +284,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     w.y = pack_bf16x2(x.z * scale, x.w * scale);
     w.z = pack_bf16x2(y.x * scale, y.y * scale);
     w.w = pack_bf16x2(y.z * scale, y.w * scale);
-    *reinterpret_cast<uint4*>(dq + b_ * sb + h_ * sh + row * sn + 8 * c8) = w;
+    *reinterpret_cast<uint4*>(dq + dq_off) = w;
   }
 }
 
@@ -378,6 +398,14 @@ __global__ void __launch_bounds__(512, 1)
   const int BH = a.B * a.H;
   const int nT = (a.N + 127) >> 7;
   const int npad = nT * 128;
+  // buffer extents for the bounds-checking build (unused otherwise)
+  const long long rows_q = VARLEN ? a.total_tokens : a.N;
+  const long long rows_k = VARLEN ? a.total_tokens : min((long long)a.N, (long long)a.kv_hi * 128) - a.kv_row_off;
+  const long long acc_lim = (long long)BH * nT * 128 * D;
+  const long long row_lim = (long long)BH * npad;
+  const long long dk_lim = extent4(VARLEN ? 1 : a.B, a.H, rows_k, D, a.dk_sb, a.dk_sh, a.dk_sn);
+  const long long dv_lim = extent4(VARLEN ? 1 : a.B, a.H, rows_k, D, a.dv_sb, a.dv_sh, a.dv_sn);
+  (void)rows_q, (void)rows_k, (void)acc_lim, (void)row_lim, (void)dk_lim, (void)dv_lim;
   // Work items are (key tile, head) pairs.  Their order groups the heads, hg
   // at a time, and within a group
   // puts the key tiles in ascending order with the group's heads interleaved:
@@ -563,10 +591,16 @@ __global__ void __launch_bounds__(512, 1)
         break;
       }
       const Item t = item_at(w);
+      if (lane == 0) {
+        (void)FA_IN(kSiteBwdItem, t.jt - kt_lo, 1, nTr, a.err);
+        (void)FA_IN(kSiteBwdItem, t.bh, 1, BH, a.err);
+        if (!SPARSE) (void)FA_IN(kSiteBwdItem, t.i_begin, t.n_steps, nT, a.err);
+      }
       if (t.n_steps == 0) continue;  // (a key tile no query tile sees loads nothing)
       auto load_kv = [&]() {
         if (lane == 0) {
           mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
+          (void)FA_IN(kSiteBwdTile, t.row0 + t.jt * 128 - a.kv_row_off, 1, rows_k, a.err);
           for (int h = 0; h < D / 64; ++h) {
             const int krow = t.row0 + t.jt * 128 - a.kv_row_off;
             tma_load_4d(smem + L::kOffK + h * L::kHalf, &tm_k, 64 * h, krow, t.hh, t.wc, bar_kv, pol_keep);
@@ -588,6 +622,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&bar_q_full[qs], L::kTile);
+          (void)FA_IN(kSiteBwdTile, t.row0 + i * 128, 1, rows_q, a.err);
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(smem + L::kOffQ + qs * L::kTile + h * L::kHalf, &tm_q, 64 * h, t.row0 + i * 128, t.hh,
                         t.wc, &bar_q_full[qs], pol_keep);
@@ -620,8 +655,10 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&bar_row_full[rs], 1024);
-          bulk_load(rowbuf, a.lse2 + (size_t)t.bh * npad + i * 128, 512, &bar_row_full[rs]);
-          bulk_load(rowbuf + 512, a.drow + (size_t)t.bh * npad + i * 128, 512, &bar_row_full[rs]);
+          long long roff = (long long)t.bh * npad + i * 128;
+          if (!FA_IN(kSiteBwdRow, roff, 128, row_lim, a.err)) roff = 0;  // (debug build: record, read row 0)
+          bulk_load(rowbuf, a.lse2 + roff, 512, &bar_row_full[rs]);
+          bulk_load(rowbuf + 512, a.drow + roff, 512, &bar_row_full[rs]);
         }
         __syncwarp();
         if (PERSIST && it == 0) {
@@ -831,7 +868,9 @@ __global__ void __launch_bounds__(512, 1)
     BitWalk walk(qbits, qbits, nwords);
     for (int it = 0; it < t.n_steps; ++it) {
       const int i = SPARSE ? walk.next() : q_tile(t, it);
-      float* tile = a.dq_acc + ((size_t)t.bh * nT + i) * (size_t)(128 * D);
+      const long long tile_off = ((long long)t.bh * nT + i) * (128 * D);
+      // (debug build: a tile outside the accumulator is recorded and tile 0 takes its adds)
+      float* tile = a.dq_acc + (FA_IN(kSiteBwdAcc, tile_off, 128 * D, acc_lim, a.err) ? tile_off : 0);
       if (L::kDqDirect) {
         if (!mbar_wait(bar_dq, (g + it) & 1, ab)) {
           ok = false;
@@ -1074,9 +1113,10 @@ __global__ void __launch_bounds__(512, 1)
     if (SPARSE && t.n_steps == 0) {
       // no query tile sees this key tile
       const long long zrow = t.row0 + key - a.kv_row_off;
-      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + zrow * a.dv_sn
-                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + zrow * a.dk_sn;
-      if (key_ok) {
+      const long long zoff = wg == 0 ? bb * a.dv_sb + hh * a.dv_sh + zrow * a.dv_sn
+                                     : bb * a.dk_sb + hh * a.dk_sh + zrow * a.dk_sn;
+      __nv_bfloat16* dst = (wg == 0 ? a.dv : a.dk) + zoff;
+      if (key_ok && FA_IN(kSiteBwdKV, zoff, D, wg == 0 ? dv_lim : dk_lim, a.err)) {
 #pragma unroll
         for (int c = 0; c < D; c += 8) st_global_v4(dst + c, 0u, 0u, 0u, 0u);
       }
@@ -1089,8 +1129,10 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t src = tmem + lane_off + (wg == 0 ? L::kColDV : L::kColDK);
       const float mul = wg == 0 ? 1.f : a.scale;
       const long long krow = t.row0 + (key_ok ? key : jt * 128) - a.kv_row_off;
-      __nv_bfloat16* dst = wg == 0 ? a.dv + bb * a.dv_sb + hh * a.dv_sh + krow * a.dv_sn
-                                   : a.dk + bb * a.dk_sb + hh * a.dk_sh + krow * a.dk_sn;
+      const long long koff = wg == 0 ? bb * a.dv_sb + hh * a.dv_sh + krow * a.dv_sn
+                                     : bb * a.dk_sb + hh * a.dk_sh + krow * a.dk_sn;
+      const bool k_in = !key_ok || FA_IN(kSiteBwdKV, koff, D, wg == 0 ? dv_lim : dk_lim, a.err);
+      __nv_bfloat16* dst = (wg == 0 ? a.dv : a.dk) + koff;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t v[32];
@@ -1099,7 +1141,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           w[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-        if (key_ok) {
+        if (key_ok && k_in) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             st_global_v4(dst + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
@@ -1185,10 +1227,10 @@ inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
   if (d == 64)
     bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                 a.scale, a.cu_seqlens, a.seqused, a.total_tokens);
+                                                 a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
   else
     bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                  a.scale, a.cu_seqlens, a.seqused, a.total_tokens);
+                                                  a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
   return cudaGetLastError();
 }
 

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -18,7 +19,15 @@
 
 namespace {
 
-__device__ int g_device_error;  // kernels record kDevTimeout / kDevMisaligned here
+// The device error word the kernels record into (kDevTimeout, kDevMisaligned,
+// kDevBadSeqlens, kDevBounds), followed by the bounds-checking build's record
+// of its first failed check: {count, site, offset, limit, block, thread}.
+struct DeviceStatus {
+  int err;
+  int pad;
+  long long rec[8];
+};
+__device__ DeviceStatus g_device_status;
 
 thread_local int t_last_cuda_error = 0;
 
@@ -81,7 +90,7 @@ bool strides_ok(const fa_strides& s) {
 
 int* device_error_ptr() {
   int* p = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess) return nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_status) != cudaSuccess) return nullptr;
   return p;
 }
 
@@ -189,10 +198,14 @@ __global__ void varlen_pad_kernel(int B, int H, int max_slot, int total, const i
     const fa_strides ss[3] = {s0, s1, s2};
     for (int k = 0; k < 3; ++k) {
       if (!ts[k]) continue;
-      __nv_bfloat16* p = ts[k] + h * ss[k].h + row * ss[k].n;
+      const long long off = h * ss[k].h + row * ss[k].n;
+      if (!FA_IN(fa::kSiteVarlenPad, off, d, fa::extent4(1, H, total, d, 0, ss[k].h, ss[k].n), &g_device_status.err))
+        continue;
+      __nv_bfloat16* p = ts[k] + off;
       for (int c = 0; c < d; c += 8) *reinterpret_cast<uint4*>(p + c) = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (lse) lse[(long long)h * total + row] = -INFINITY;
+    if (lse && FA_IN(fa::kSiteVarlenPad, (long long)h * total + row, 1, (long long)H * total, &g_device_status.err))
+      lse[(long long)h * total + row] = -INFINITY;
   }
 }
 
@@ -255,14 +268,41 @@ const char* fa_strerror(int status) {
 
 int fa_last_cuda_error(void) { return t_last_cuda_error; }
 
+int fa_debug_bounds_record(long long* out, void* stream) {
+  if (!out) return FA_ERR_INVALID_ARG;
+#ifdef FA_DEBUG
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  long long rec[8];
+  e = cudaMemcpyFromSymbol(rec, g_device_status, sizeof(rec), offsetof(DeviceStatus, rec));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const long long zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  e = cudaMemcpyToSymbol(g_device_status, zero, sizeof(zero), offsetof(DeviceStatus, rec));
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int i = 0; i < 6; ++i) out[i] = rec[i];
+  return FA_OK;
+#else
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;
+#endif
+}
+
+int fa_debug_build(void) {
+#ifdef FA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 int fa_get_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e);
   int value = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&value, g_device_error, sizeof(int));
+  e = cudaMemcpyFromSymbol(&value, g_device_status, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e);
   return value;
 }

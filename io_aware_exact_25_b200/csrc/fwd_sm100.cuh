@@ -45,6 +45,7 @@
 // stale m, so the final O / l is exact; P values stay below 256.
 #pragma once
 
+#include "debug_check.cuh"
 #include "dropout_hash.cuh"
 #include "sm100.cuh"
 
@@ -162,6 +163,13 @@ __global__ void __launch_bounds__(320, 1)
   }
   const int n_kv_all = (seq_len + 127) >> 7;
   const int qt0 = 2 * cta_tile;
+  // buffer extents for the bounds-checking build (unused otherwise)
+  const long long rows_q = VARLEN ? a.total_tokens : a.N;
+  const long long rows_k = VARLEN ? a.total_tokens : min((long long)a.N, (long long)a.kv_hi * 128) - a.kv_row_off;
+  const long long o_lim = extent4(VARLEN ? 1 : a.B, a.H, rows_q, D, a.o_sb, a.o_sh, a.o_sn);
+  const long long lse_lim = VARLEN ? (long long)a.H * a.total_tokens : (long long)BH * a.N;
+  const long long part_rows = (long long)a.num_splits * BH * a.N;
+  (void)rows_q, (void)rows_k, (void)o_lim, (void)lse_lim, (void)part_rows;
   const bool act1 = (qt0 + 1) * 128 < seq_len;
   // key tiles each Q tile sees: [0, end_t)
   const int end0 = CAUSAL ? qt0 + 1 : n_kv_all;
@@ -242,6 +250,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < 2 && nkv_max > 0; ++t) {
         if (t == 1 && !act1) break;
         mbar_arrive_expect_tx(&bar_q[t], L::kTile);
+        (void)FA_IN(kSiteFwdTile, row0 + (qt0 + t) * 128, 1, rows_q, a.err);
         for (int h = 0; h < D / 64; ++h)
           tma_load_4d(smem + L::kOffQ + t * L::kTile + h * L::kHalf, &tm_q, 64 * h, row0 + (qt0 + t) * 128, hh,
                       wc, &bar_q[t], pol_once);
@@ -260,6 +269,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
+          (void)FA_IN(kSiteFwdTile, row0 + kt * 128 - a.kv_row_off, 1, rows_k, a.err);
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h,
                         row0 + kt * 128 - a.kv_row_off, hh, wc, &bar_kv_full[stage], pol_keep);
@@ -523,30 +533,36 @@ __global__ void __launch_bounds__(320, 1)
       if (SPARSE && nkv == 0) {
         // the mask hides every key tile from this query tile
         if (in_range && ok) {
-          __nv_bfloat16* orow = a.o + bb * a.o_sb + hh * a.o_sh + (long long)q_row * a.o_sn;
+          const long long ooff = bb * a.o_sb + hh * a.o_sh + (long long)q_row * a.o_sn;
+          __nv_bfloat16* orow = a.o + ooff;
+          if (FA_IN(kSiteFwdO, ooff, D, o_lim, a.err)) {
 #pragma unroll
-          for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
-          a.lse[lse_base + q_row] = -INFINITY;
+            for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+          }
+          if (FA_IN(kSiteFwdLse, lse_base + q_row, 1, lse_lim, a.err)) a.lse[lse_base + q_row] = -INFINITY;
         }
       } else if (SPLIT && nkv == 0) {
         // this split holds no key tile of this query tile: an empty partial
-        if (in_range && ok) {
-          float* prow = a.part_o + (((size_t)split * BH + bh) * a.N + q_row) * D;
+        const long long prow_i = ((long long)split * BH + bh) * a.N + q_row;
+        if (in_range && ok && FA_IN(kSiteFwdPart, prow_i, 1, part_rows, a.err)) {
+          float* prow = a.part_o + prow_i * D;
 #pragma unroll
           for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(prow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-          a.part_lse[((size_t)split * BH + bh) * a.N + q_row] = -INFINITY;
+          a.part_lse[prow_i] = -INFINITY;
         }
       } else if (ok && mbar_wait(&bar_pv[t], (nkv - 1) & 1, ab)) {
         tc_fence_after();
         const float inv_l = 1.f / l;
         const float lse_row = (m_used + log2f(l)) * 0.69314718055994531f;
         if (SPLIT) {
-          float* prow = a.part_o + (((size_t)split * BH + bh) * a.N + (size_t)(in_range ? q_row : 0)) * D;
+          const long long prow_i = ((long long)split * BH + bh) * a.N + (in_range ? q_row : 0);
+          const bool p_ok = FA_IN(kSiteFwdPart, prow_i, 1, part_rows, a.err);
+          float* prow = a.part_o + prow_i * D;
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t o[32];
             tmem_ld32_sync(tO + 32u * c4, o);
-            if (in_range) {
+            if (in_range && p_ok) {
 #pragma unroll
               for (int v4 = 0; v4 < 8; ++v4)
                 *reinterpret_cast<float4*>(prow + 32 * c4 + 4 * v4) =
@@ -554,10 +570,11 @@ __global__ void __launch_bounds__(320, 1)
                                 __uint_as_float(o[4 * v4 + 2]) * inv_l, __uint_as_float(o[4 * v4 + 3]) * inv_l);
             }
           }
-          if (in_range) a.part_lse[((size_t)split * BH + bh) * a.N + q_row] = lse_row;
+          if (in_range && p_ok) a.part_lse[prow_i] = lse_row;
         } else {
-          __nv_bfloat16* orow =
-              a.o + bb * a.o_sb + hh * a.o_sh + (long long)(row0 + (in_range ? q_row : 0)) * a.o_sn;
+          const long long ooff = bb * a.o_sb + hh * a.o_sh + (long long)(row0 + (in_range ? q_row : 0)) * a.o_sn;
+          const bool o_ok = FA_IN(kSiteFwdO, ooff, D, o_lim, a.err);
+          __nv_bfloat16* orow = a.o + ooff;
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t o[32];
@@ -566,13 +583,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k)
               w[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
-            if (in_range) {
+            if (in_range && o_ok) {
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4)
                 st_global_v4(orow + 32 * c4 + 8 * v4, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
             }
           }
-          if (in_range) a.lse[lse_base + q_row] = lse_row;
+          if (in_range && FA_IN(kSiteFwdLse, lse_base + q_row, 1, lse_lim, a.err)) a.lse[lse_base + q_row] = lse_row;
         }
       }
     }
@@ -597,7 +614,11 @@ __global__ void __launch_bounds__(256) splitkv_combine_kernel(const FwdArgs a) {
   const int lane = threadIdx.x & 31;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const long long o_lim = extent4(a.B, a.H, a.N, D, a.o_sb, a.o_sh, a.o_sn);
+  (void)o_lim;
   for (long long r = warp0; r < rows; r += nwarps) {
+    if (!FA_IN(kSiteCombine, (long long)(a.num_splits - 1) * rows + r, 1, (long long)a.num_splits * rows, a.err))
+      continue;
     float mx = -INFINITY;
     for (int s = 0; s < a.num_splits; ++s) mx = fmaxf(mx, a.part_lse[(size_t)s * rows + r]);
     float acc[kPer];
@@ -615,7 +636,9 @@ __global__ void __launch_bounds__(256) splitkv_combine_kernel(const FwdArgs a) {
     const float inv = 1.f / wsum;
     const int bh = (int)(r / a.N), i = (int)(r - (long long)bh * a.N);
     const int b_ = bh / a.H, h_ = bh - b_ * a.H;
-    __nv_bfloat16* orow = a.o + b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn + lane * kPer;
+    const long long ooff = b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn;
+    if (!FA_IN(kSiteCombine, ooff, D, o_lim, a.err)) continue;
+    __nv_bfloat16* orow = a.o + ooff + lane * kPer;
 #pragma unroll
     for (int e = 0; e < kPer; e += 2) *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
     if (lane == 0) a.lse[r] = mx + logf(wsum);

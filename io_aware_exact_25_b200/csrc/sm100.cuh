@@ -18,6 +18,7 @@ enum : int {
   kDevTimeout = 1,      // a bounded mbarrier wait ran out
   kDevMisaligned = 2,   // shared-memory tile base not 1024-byte aligned
   kDevBadSeqlens = 3,   // variable-length offsets or lengths out of range (clamped)
+  kDevBounds = 4,       // a bounds check failed (bounds-checking build only)
 };
 
 // Upper bound on any single wait (ns).  Kernels here run for milliseconds;

@@ -36,6 +36,18 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(binding.EXPORTS) == set(names)
 
 
+def test_bounds_checking_build_exports_the_same_symbols(lib):
+    """libfa_sm100_debug.so (FA_DEBUG) is the same ABI with its checks on;
+    only it answers the record query (no device is touched for either)."""
+    dbg = ctypes.CDLL(binding.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    assert lib.fa_debug_build() == 0 and dbg.fa_debug_build() == 1
+    out = (ctypes.c_longlong * 6)()
+    assert lib.fa_debug_bounds_record(out, None) == binding.FA_ERR_UNSUPPORTED
+    assert dbg.fa_debug_bounds_record(None, None) == binding.FA_ERR_INVALID_ARG
+
+
 def test_status_codes_match_header(lib):
     text = open(os.path.join(ROOT, "include", "fa.h")).read()
     codes = dict((k, int(v)) for k, v in re.findall(r"(FA_[A-Z_]+)\s*=\s*(-?\d+)", text))
