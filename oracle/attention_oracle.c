@@ -16,7 +16,7 @@
  *   l_i   = sum_j exp(s_ij - m_i)
  *   P_ij  = exp(s_ij - m_i) / l_i
  *   lse_i = m_i + ln(l_i)
- *   Z_ij  = [hash32(seed,b,h,i,j) >= T]   ; T = ceil(p * 2^32), p=0 keeps all
+ *   Z_ij  = [h16(i,j) >= T]                ; T = ceil(p * 2^16), p=0 keeps all
  *   Pd_ij = P_ij * Z_ij / (1 - p)          (dropout applied after softmax)
  *   O_i   = sum_j Pd_ij v_j
  *
@@ -124,8 +124,12 @@ static double dot_rows(row_t a, row_t b, int d) {
  *   C1 = floor(frac(sqrt 2) * 2^32), C2 = floor(frac(sqrt 3) * 2^32),
  *   G  = floor(2^32 / golden ratio)
  *   row key  k_i = mix(mix(mix(mix(mix(lo(seed)^G) ^ hi(seed)) ^ b) ^ h) ^ i)
- *   element  hash32(seed,b,h,i,j) = mix(k_i ^ (j*G))
- *   keep iff hash32 >= T, T = ceil(p * 2^32).
+ *   pair     hash32(seed,b,h,i,u) = mix(k_i ^ (u*G)), u = j >> 1: one mix
+ *            decides the two adjacent keys 2u and 2u+1 of row i
+ *   element  h16(i,j) = low 16 bits of hash32(.., i, j >> 1) for even j,
+ *            high 16 bits for odd j
+ *   keep iff h16 >= T, T = ceil(p * 2^16) (0 <= T <= 2^16), so the keep
+ *   probability (2^16 - T) / 2^16 is within 2^-16 of 1 - p.
  * The constants are derived here from their definitions, not typed in.
  */
 static uint32_t C1, C2, G;
@@ -166,18 +170,20 @@ uint32_t orc_hash32(uint64_t seed, uint32_t b, uint32_t h, uint32_t i, uint32_t 
     return mix32(key ^ (j * G));
 }
 
-/* T = ceil(p * 2^32) as an unsigned 32-bit threshold; p in [0, 1). */
+/* T = ceil(p * 2^16), compared with 16-bit hash halves; p in [0, 1). */
 uint32_t orc_keep_threshold(double p) {
-    double t = ceil(p * 4294967296.0);
+    double t = ceil(p * 65536.0);
     if (t <= 0.0) return 0u;
-    if (t >= 4294967295.0) return 4294967295u;
+    if (t >= 65536.0) return 65536u;
     return (uint32_t)t;
 }
 
 static int keep_elem(const problem_t *pb, int bh, int i, int j) {
     if (pb->p_drop <= 0.0) return 1;
     uint32_t b = (uint32_t)(bh / pb->H), h = (uint32_t)(bh % pb->H);
-    return orc_hash32(pb->seed, b, h, (uint32_t)i, (uint32_t)j) >= orc_keep_threshold(pb->p_drop);
+    uint32_t w = orc_hash32(pb->seed, b, h, (uint32_t)i, (uint32_t)j >> 1);
+    uint32_t h16 = (j & 1) ? (w >> 16) : (w & 0xffffu);
+    return h16 >= orc_keep_threshold(pb->p_drop);
 }
 
 /* -------------------------------------------------------- one query row */

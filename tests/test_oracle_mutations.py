@@ -37,7 +37,8 @@ MUTANTS = {
     "empty_row_lse_zero": ("*lse = l > 0.0 ? m + log(l) : -INFINITY;", "*lse = l > 0.0 ? m + log(l) : 0.0;"),
     "hash_constant_typo": ("C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32);",
                            "C2 = (uint32_t)(uint64_t)floor((sqrt(3.0) - 1.0) * two32) + 2u;"),
-    "threshold_floor": ("double t = ceil(p * 4294967296.0);", "double t = floor(p * 4294967296.0);"),
+    "threshold_floor": ("double t = ceil(p * 65536.0);", "double t = floor(p * 65536.0);"),
+    "pair_same_half": ("uint32_t h16 = (j & 1) ? (w >> 16) : (w & 0xffffu);", "uint32_t h16 = w & 0xffffu;"),
 }
 
 

@@ -53,10 +53,30 @@ def test_hash_constants_match_published_values():
 
 def test_keep_threshold_closed_forms():
     assert oracle.keep_threshold(0.0) == 0
-    assert oracle.keep_threshold(0.5) == 2 ** 31
-    # ceil(0.1 * 2^32) = ceil(429496729.6)
-    assert oracle.keep_threshold(0.1) == 429496730
-    assert oracle.keep_threshold(0.25) == 2 ** 30
+    assert oracle.keep_threshold(0.5) == 2 ** 15
+    # ceil(0.1 * 2^16) = ceil(6553.6)
+    assert oracle.keep_threshold(0.1) == 6554
+    assert oracle.keep_threshold(0.25) == 2 ** 14
+    # the largest p below 1 keeps nothing: T = 2^16 exceeds every 16-bit half
+    assert oracle.keep_threshold(1.0 - 2.0 ** -20) == 2 ** 16
+
+
+def test_adjacent_keys_use_independent_halves():
+    """Keys 2u and 2u+1 of a row share one 32-bit mix but read disjoint
+    halves of it: their keep decisions must be uncorrelated (a mask that
+    read the same half, or the same bits, for both would make them equal),
+    and the pair's keep rate must be (1 - p)^2."""
+    p = 0.3
+    mask = oracle.dropout_mask(1, 2, 1024, p, seed=8).astype(np.float64)
+    even, odd = mask[..., 0::2].ravel(), mask[..., 1::2].ravel()
+    n = even.size
+    corr = np.corrcoef(even, odd)[0, 1]
+    assert abs(corr) < 5 / math.sqrt(n)
+    both = (even * odd).mean()
+    assert abs(both - (1 - p) ** 2) < 5 * math.sqrt((1 - p) ** 2 * (1 - (1 - p) ** 2) / n)
+    # and every key's rate on its own is 1 - p
+    for half in (even, odd):
+        assert abs(half.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
 
 
 def test_dropout_mask_statistics():
