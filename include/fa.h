@@ -22,8 +22,10 @@
  *    launches nothing (pointers are then not inspected).
  *  - scale > 0 and finite (1/sqrt(d) is the usual choice).  causal is 0 or 1:
  *    query i sees keys j <= i.  dropout_p in [0, 1): element (i, j) of head
- *    (b, h) is kept iff hash32(seed, b, h, i, j) >= ceil(dropout_p * 2^32)
- *    (hash32 is defined in io_aware_exact_25_b200/csrc/dropout_hash.cuh);
+ *    (b, h) is kept iff the 16-bit half h16(i, j) of the 32-bit mix
+ *    hash32(seed, b, h, i, j >> 1) -- the low half for even j, the high half
+ *    for odd j -- is >= ceil(dropout_p * 2^16) (both are defined in
+ *    io_aware_exact_25_b200/csrc/dropout_hash.cuh);
  *    kept probabilities are scaled by 1/(1-p).
  *    Dropout is applied after the softmax, so lse is that of the undropped
  *    scores.  The backward with the same (seed, dropout_p) regenerates the

@@ -1014,15 +1014,29 @@ __global__ void __launch_bounds__(512, 1)
       }
       uint32_t keep_bits[2] = {0xffffffffu, 0xffffffffu};
       if (DROPOUT) {
+        // Key pair u = key >> 1 is decided by one hash per query; the even
+        // key reads its low 16 bits and the odd key its high 16 bits:
+        // (w & 0xffff) >= T for the even key, and w >= T * 2^16, which is
+        // (w >> 16) >= T, for the odd key -- one mask and one compare.
+        // (Sharing each hash between the two lanes of a pair by a shuffle was
+        // measured at twice the kernel time.)
+        const bool odd = (jr & 1) != 0;
+        const uint32_t u = (uint32_t)key >> 1;
+        const uint32_t lane_mask = odd ? 0xffffffffu : 0xffffu;
+        const uint32_t lane_thr = odd ? (a.drop_threshold << 16) : a.drop_threshold;
+        if (a.drop_threshold >= 65536u) {
+          keep_bits[0] = keep_bits[1] = 0u;  // p so close to 1 that every element is dropped
+        } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 k4 = ld_shared_f4(rowbuf + 1024u + 4u * (col0 + 4 * c4));
-          const uint32_t kv[4] = {__float_as_uint(k4.x), __float_as_uint(k4.y), __float_as_uint(k4.z),
-                                  __float_as_uint(k4.w)};
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 k4 = ld_shared_f4(rowbuf + 1024u + 4u * (col0 + 4 * c4));
+            const uint32_t kv[4] = {__float_as_uint(k4.x), __float_as_uint(k4.y), __float_as_uint(k4.z),
+                                    __float_as_uint(k4.w)};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            if (dropout_hash(kv[e], (uint32_t)key) < a.drop_threshold) keep_bits[c >> 5] &= ~(1u << (c & 31));
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * c4 + e;
+              if ((dropout_hash(kv[e], u) & lane_mask) < lane_thr) keep_bits[c >> 5] &= ~(1u << (c & 31));
+            }
           }
         }
       }

@@ -8,9 +8,11 @@
 //   C2 = floor(frac(sqrt 3) * 2^32) = 0xbb67ae85
 //   G  = floor(2^32 / golden ratio) = 0x9e3779b9
 //   row key   k_i = mix(mix(mix(mix(mix(lo32(seed) ^ G) ^ hi32(seed)) ^ b) ^ h) ^ i)
-//   element   hash32(seed, b, h, i, j) = mix(k_i ^ (j * G))
-// Element (i, j) of head (b, h) is kept iff hash32 >= T with
-// T = ceil(p * 2^32) computed on the host in double precision; survivors are
+//   pair      hash32(seed, b, h, i, u) = mix(k_i ^ (u * G)), u = j >> 1
+// One mix decides the two adjacent keys 2u and 2u+1 of row i: element (i, j)
+// of head (b, h) is kept iff its 16-bit half -- the low half of the pair's
+// hash for even j, the high half for odd j -- is >= T, T = ceil(p * 2^16)
+// computed on the host in double precision (0 <= T <= 2^16); survivors are
 // scaled by 1/(1-p).  The mask is applied after the softmax, so the row sums
 // and the logsumexp use the undropped probabilities.
 #pragma once
@@ -41,8 +43,13 @@ __host__ __device__ __forceinline__ uint32_t dropout_row_key(uint64_t seed, uint
   return mix32(k ^ i);
 }
 
-__host__ __device__ __forceinline__ uint32_t dropout_hash(uint32_t row_key, uint32_t j) {
-  return mix32(row_key ^ (j * kGolden));
+// the hash of key pair u = j >> 1 of a row
+__host__ __device__ __forceinline__ uint32_t dropout_hash(uint32_t row_key, uint32_t u) {
+  return mix32(row_key ^ (u * kGolden));
 }
+
+// keep decisions of the pair's even key (low half) and odd key (high half)
+__host__ __device__ __forceinline__ bool keep_lo(uint32_t w, uint32_t threshold) { return (w & 0xffffu) >= threshold; }
+__host__ __device__ __forceinline__ bool keep_hi(uint32_t w, uint32_t threshold) { return (w >> 16) >= threshold; }
 
 }  // namespace fa

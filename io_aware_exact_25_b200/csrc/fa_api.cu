@@ -113,10 +113,11 @@ int check_common(int B, int H, int N, int d, float scale, int causal, float drop
   return FA_OK;
 }
 
+// T = ceil(p * 2^16), compared with the 16-bit halves of the pair hash
 uint32_t keep_threshold(float p) {
-  const double t = std::ceil((double)p * 4294967296.0);
+  const double t = std::ceil((double)p * 65536.0);
   if (t <= 0.0) return 0u;
-  if (t >= 4294967295.0) return 4294967295u;
+  if (t >= 65536.0) return 65536u;
   return (uint32_t)t;
 }
 
@@ -174,7 +175,8 @@ __global__ void dropout_mask_kernel(int H, int N, uint32_t threshold, uint64_t s
     const int hi = (int)(hr / nrows);
     const int bh = heads[hi];
     const uint32_t key = fa::dropout_row_key(seed, (uint32_t)(bh / H), (uint32_t)(bh % H), (uint32_t)rows[ri]);
-    out[u] = fa::dropout_hash(key, (uint32_t)j) >= threshold ? 1 : 0;
+    const uint32_t w = fa::dropout_hash(key, (uint32_t)j >> 1);
+    out[u] = ((j & 1) ? fa::keep_hi(w, threshold) : fa::keep_lo(w, threshold)) ? 1 : 0;
   }
 }
 

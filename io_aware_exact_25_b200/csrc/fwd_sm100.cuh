@@ -54,7 +54,7 @@ namespace fa {
 struct FwdArgs {
   int B, H, N;
   float scale_log2;         // scale * log2(e)
-  uint32_t drop_threshold;  // keep iff hash32 >= threshold
+  uint32_t drop_threshold;  // keep iff the key's 16-bit half of the pair hash >= threshold
   float drop_scale;         // 1 / (1 - p)
   uint64_t seed;
   __nv_bfloat16* o;            // [B,H,N,D] with element strides o_sb, o_sh, o_sn
@@ -500,9 +500,10 @@ __global__ void __launch_bounds__(320, 1)
           }
           sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
           if (DROPOUT) {
-            const uint32_t col = (uint32_t)(jg * 128 + 2 * c);
-            p0 = dropout_hash(rkey, col) >= a.drop_threshold ? p0 * a.drop_scale : 0.f;
-            p1 = dropout_hash(rkey, col + 1) >= a.drop_threshold ? p1 * a.drop_scale : 0.f;
+            // keys 2c and 2c+1 of the tile: one pair hash
+            const uint32_t w = dropout_hash(rkey, (uint32_t)(jg * 64 + c));
+            p0 = keep_lo(w, a.drop_threshold) ? p0 * a.drop_scale : 0.f;
+            p1 = keep_hi(w, a.drop_threshold) ? p1 * a.drop_scale : 0.f;
           }
           pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
           if (c == 31) {
