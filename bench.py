@@ -269,6 +269,60 @@ def workload_config(w, mask_kind=None, frac=None):
 
 # ------------------------------------------------------------ our arm
 
+def pipelined_e2e(dev, stream, x, d_in0, d_out0, compute, steps, barrier):
+    """End to end through the public API: every step copies its inputs from
+    pinned host memory to the device, runs ``compute(inputs, outputs,
+    stream)`` and copies every result back.  Uploads, compute and downloads
+    run on three streams over two sets of device buffers, so step k+1's
+    upload and step k-1's download overlap step k's compute (the PCIe link is
+    full duplex).  Returns (ms for ``steps`` steps, H2D and D2H bytes a step)."""
+    import torch
+    h_in = {n: x[n].pin_memory() for n in d_in0}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    nbuf = 2
+    d_in = [d_in0] + [{n: torch.empty_like(t) for n, t in d_in0.items()} for _ in range(nbuf - 1)]
+    d_out = [d_out0] + [{n: torch.empty_like(t) for n, t in d_out0.items()} for _ in range(nbuf - 1)]
+    h_out = [{n: torch.empty_like(t, device="cpu").pin_memory() for n, t in d_out0.items()} for _ in range(nbuf)]
+    d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
+    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_cmp = stream
+    ev_up, ev_cmp, ev_dn = ([torch.cuda.Event() for _ in range(nbuf)] for _ in range(3))
+    for evs, st in ((ev_up, s_up), (ev_cmp, s_cmp), (ev_dn, s_dn)):
+        for e in evs:
+            e.record(st)
+
+    def step(kstep):
+        bi = kstep % nbuf
+        din, dout, hout = d_in[bi], d_out[bi], h_out[bi]
+        s_up.wait_event(ev_cmp[bi])  # step k-2 finished reading these inputs
+        with torch.cuda.stream(s_up):
+            for n, h in h_in.items():
+                din[n].copy_(h, non_blocking=True)
+        ev_up[bi].record(s_up)
+        s_cmp.wait_event(ev_up[bi])
+        s_cmp.wait_event(ev_dn[bi])  # step k-2's results are on the host
+        compute(din, dout, s_cmp)
+        ev_cmp[bi].record(s_cmp)
+        s_dn.wait_event(ev_cmp[bi])
+        with torch.cuda.stream(s_dn):
+            for n, t in dout.items():
+                hout[n].copy_(t, non_blocking=True)
+        ev_dn[bi].record(s_dn)
+
+    for kstep in range(3):
+        step(kstep)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_up)
+    for kstep in range(steps):
+        step(kstep)
+    e1.record(s_dn)  # the last download follows every upload and every compute
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1), h2d, d2h
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -396,58 +450,16 @@ def run_ours(args, w):
     # copies every result back.  Uploads, compute and downloads run on three
     # streams over two sets of device buffers, so step k+1's upload and step
     # k-1's download overlap step k's compute (the PCIe link is full duplex).
-    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    nbuf = 2
-    d_in = [{"q": q, "k": k, "v": v, "do": do}] + [
-        {n: torch.empty_like(q) for n in ("q", "k", "v", "do")} for _ in range(nbuf - 1)]
-    d_out = [{"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}] + [
-        {"o": torch.empty_like(q), "lse": torch.empty_like(lse), "dq": torch.empty_like(q),
-         "dk": torch.empty_like(q), "dv": torch.empty_like(q)} for _ in range(nbuf - 1)]
-    h_out = [{n: torch.empty_like(t, device="cpu").pin_memory() for n, t in d_out[0].items()} for _ in range(nbuf)]
-    d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
-    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    s_cmp = stream
-    ev_up, ev_cmp, ev_dn = ([torch.cuda.Event() for _ in range(nbuf)] for _ in range(3))
-    for evs, st in ((ev_up, s_up), (ev_cmp, s_cmp), (ev_dn, s_dn)):
-        for e in evs:
-            e.record(st)
-
-    def e2e_step(kstep):
-        bi = kstep % nbuf
-        din, dout, hout = d_in[bi], d_out[bi], h_out[bi]
-        s_up.wait_event(ev_cmp[bi])  # step k-2 finished reading these inputs
-        with torch.cuda.stream(s_up):
-            for n, h in (("q", hq), ("k", hk), ("v", hv), ("do", hdo)):
-                din[n].copy_(h, non_blocking=True)
-        ev_up[bi].record(s_up)
-        s_cmp.wait_event(ev_up[bi])
-        s_cmp.wait_event(ev_dn[bi])  # step k-2's results are on the host
+    def compute(din, dout, st):
         binding.fwd(din["q"], din["k"], din["v"], causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
-                    o=dout["o"], lse=dout["lse"], block_mask=mask, stream=s_cmp)
+                    o=dout["o"], lse=dout["lse"], block_mask=mask, stream=st)
         binding.bwd(din["q"], din["k"], din["v"], dout["o"], din["do"], dout["lse"], causal=w.causal, scale=w.scale,
                     dropout_p=w.p_drop, seed=w.seed, dq=dout["dq"], dk=dout["dk"], dv=dout["dv"], workspace=work,
-                    block_mask=mask, stream=s_cmp)
-        ev_cmp[bi].record(s_cmp)
-        s_dn.wait_event(ev_cmp[bi])
-        with torch.cuda.stream(s_dn):
-            for n, t in dout.items():
-                hout[n].copy_(t, non_blocking=True)
-        ev_dn[bi].record(s_dn)
+                    block_mask=mask, stream=st)
 
     e2e_steps = max(3, min(args.steps, 20))
-    for kstep in range(3):
-        e2e_step(kstep)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_up)
-    for kstep in range(e2e_steps):
-        e2e_step(kstep)
-    e1.record(s_dn)  # the last download follows every upload and every compute
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, x, {"q": q, "k": k, "v": v, "do": do},
+                                     {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}, compute, e2e_steps, barrier)
     if binding.device_error(stream) != 0:
         raise RuntimeError("kernel reported a device error in the end-to-end run")
 
@@ -658,32 +670,24 @@ def run_ours_varlen(args, w):
     ok = ok and bool((seg_sum(dk).abs() <= 1e-2 * seg_sum(dk.abs()) + 1e-2).all())
     if w.p_drop == 0.0:
         ok = ok and bool(((seg_sum(dv) - seg_sum(do)).abs() <= 1e-2 * seg_sum(dv.abs()) + 1e-2).all())
-    # end to end through the public API: pinned host inputs in, results out
-    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
-    h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (o, lse, dq, dk, dv)]
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    # end to end through the public API, inputs from and results to pinned
+    # host memory (the same three-stream pipeline as the dense path)
+    def compute(din, dout, st):
+        binding.fwd_varlen(din["q"], din["k"], din["v"], cu, maxs, causal=w.causal, scale=w.scale,
+                           dropout_p=w.p_drop, seed=w.seed, o=dout["o"], lse=dout["lse"], stream=st)
+        binding.bwd_varlen(din["q"], din["k"], din["v"], dout["o"], din["do"], dout["lse"], cu, maxs,
+                           causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed, dq=dout["dq"],
+                           dk=dout["dk"], dv=dout["dv"], workspace=work, stream=st)
 
-    def e2e_step():
-        for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
-            dst.copy_(src, non_blocking=True)
-        binding.fwd_varlen(q, k, v, cu, maxs, causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed,
-                           o=o, lse=lse)
-        binding.bwd_varlen(q, k, v, o, do, lse, cu, maxs, causal=w.causal, scale=w.scale, dropout_p=w.p_drop,
-                           seed=w.seed, dq=dq, dk=dk, dv=dv, workspace=work)
-        for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
-            dst.copy_(src, non_blocking=True)
+    def barrier():
+        if ws > 1:
+            dist.barrier()
 
-    e2e_steps = max(3, min(args.steps, 10))
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms, h2d, d2h = pipelined_e2e(dev, stream, x, {"q": q, "k": k, "v": v, "do": do},
+                                     {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}, compute, e2e_steps, barrier)
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error in the end-to-end run")
     from io_aware_exact_25_b200.replicas import replica_summary
     summ = replica_summary(elapsed_ms, e2e_ms, stage_ms, ok, device=dev)
     if not summ["all_ok"]:
@@ -725,7 +729,8 @@ def run_ours_varlen(args, w):
                              "sample": f"fp64 fwd+bwd of sequence 0 (first {L0} tokens), head 0 ({cpu_dt:.1f} s)"},
             "e2e": {"value": ws * (ff + fb) * e2e_steps / (summ["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "binding.fwd_varlen/binding.bwd_varlen (C ABI) with pinned host buffers, one stream"},
+                    "api": "binding.fwd_varlen/binding.bwd_varlen (C ABI) with pinned host buffers; uploads, "
+                           "compute and downloads on three streams over two device buffer sets"},
             "gpu_launches": args.steps * (1 + 3),
             "replica_checks": {"ranks": ws, "all_ok": summ["all_ok"],
                                "checks": "finite outputs; per sequence and head sum_j dK_j = 0 and "
