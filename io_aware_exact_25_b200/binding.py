@@ -58,12 +58,13 @@ class FaError(RuntimeError):
 
 def load() -> ctypes.CDLL:
     """Load ``libfa_sm100.so`` (raises if it has not been built); every
-    function of this module calls through it."""
+    function of this module calls through it.  With ``FA_BOUNDS_CHECK=1`` in
+    the environment the bounds-checking build is loaded instead."""
     global _lib
     with _lock:
         if _lib is not None:
             return _lib
-        _lib = _open(LIB_PATH)
+        _lib = _open(DEBUG_LIB_PATH if os.environ.get("FA_BOUNDS_CHECK") == "1" else LIB_PATH)
         return _lib
 
 

@@ -29,6 +29,25 @@ def _parity_test_id(request):
     yield
 
 
+@pytest.fixture(autouse=True)
+def _bounds_record(request):
+    """With FA_BOUNDS_CHECK=1 the whole suite runs on the bounds-checking
+    build: after every GPU test its record of failed checks must be empty."""
+    yield
+    if os.environ.get("FA_BOUNDS_CHECK") != "1" or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    from io_aware_exact_25_b200 import binding
+    lib = binding.load()
+    if lib.fa_debug_build() != 1:
+        return  # a test swapped in another build and has not restored it
+    rec = binding.debug_bounds_record()
+    assert rec[0] == 0, (f"bounds check failed: site {rec[1]}, offset {rec[2]}, limit {rec[3]}, block {rec[4]}, "
+                         f"thread {rec[5]} ({rec[0]} failures)")
+
+
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
     """Print every use of the parity bar's recorded exception (elements above
     2e-2 that the |ref| >= 4 rounding allowance admits)."""
