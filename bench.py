@@ -420,8 +420,12 @@ def run_ours(args, w):
     t_start.record(stream)
     for st in range(args.steps):
         ev[st][0].record(stream)
-        for i, (_, fn) in enumerate(stages):
+        for i, (name, fn) in enumerate(stages):
+            if args.nvtx:
+                torch.cuda.nvtx.range_push(name)
             fn()
+            if args.nvtx:
+                torch.cuda.nvtx.range_pop()
             ev[st][i + 1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -646,8 +650,12 @@ def run_ours_varlen(args, w):
     t0.record(stream)
     for st in range(args.steps):
         ev[st][0].record(stream)
-        for i, (_, fn) in enumerate(stages):
+        for i, (name, fn) in enumerate(stages):
+            if args.nvtx:
+                torch.cuda.nvtx.range_push(name)
             fn()
+            if args.nvtx:
+                torch.cuda.nvtx.range_pop()
             ev[st][i + 1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
@@ -760,6 +768,8 @@ def main():
     ap.add_argument("--block-mask", default=None,
                     help="block-sparse run with this synthetic block mask, e.g. 'local:4,global:2' or "
                          "'random:0.25' (io_aware_exact_25_b200.inputs.block_mask)")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="wrap each stage launch of the timed region in an NVTX range (for profiler timelines)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end and CPU-baseline legs (profiling runs)")
     ap.add_argument("--ref-rows", type=int, default=1024,
