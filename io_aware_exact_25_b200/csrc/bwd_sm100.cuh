@@ -295,12 +295,17 @@ struct BwdLayout {
   // 16 warps: P/dS warpgroups 0-1, dQ warpgroup 2, and warpgroup 3 (MMA
   // issue, TMA producer, two idle warps) so that every warpgroup is whole for
   // the register reallocation: launched at 128 registers a thread (the whole
-  // register file), then 160 for the P/dS warpgroups, 104 for dQ and 80 for
-  // warpgroup 3 -- 2*4*32*160 + 4*32*104 + 4*32*80 = 64512 <= 65536.  (At 128
-  // registers for every warp the dropout kernels spilled 220-280 bytes a
-  // thread; with this split 12.)
+  // register file), then for the P/dS warpgroups, dQ and warpgroup 3
+  // 152 / 112 / 88 without dropout and 160 / 104 / 80 with it (both sum to
+  // 2*128*R_ps + 128*R_dq + 128*R_ctl = 64512 <= 65536).  At 128 registers
+  // for every warp the dropout kernels spilled 220-280 bytes a thread; with
+  // these splits none of the kernels without dropout spills (the long8k
+  // backward 1.7 % faster than at 160/104/80, which spilled 48 bytes) and the
+  // dropout kernels spill 0-12 (160/112/72 spills 4 there but measured 1 %
+  // slower on long64k).
   static constexpr int kThreads = 512;
-  static constexpr uint32_t kRegsPS = 160, kRegsDQ = 104, kRegsCtl = 80;
+  static constexpr uint32_t kRegsPS = DROPOUT ? 160 : 152, kRegsDQ = DROPOUT ? 104 : 112,
+                            kRegsCtl = DROPOUT ? 80 : 88;
   static_assert(2 * 128 * kRegsPS + 128 * kRegsDQ + 128 * kRegsCtl <= 512 * 128, "register split");
   static constexpr uint32_t kHalf = 128u * 128u;
   static constexpr uint32_t kTile = 128u * D * 2u;
