@@ -59,14 +59,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tensor map of a bf16 [B, H, N, d] tensor with element strides s (d
-// contiguous), addressed as {d, n, h, b} and read in 128-row x 64-column boxes
-// with the 128-byte swizzle; rows past N read as zero.
-int make_tile_map(CUtensorMap* m, const void* base, int B, int H, int N, int d, const fa_strides& s) {
+// contiguous), addressed as {d, n, h, b} and read in box_rows-row x 64-column
+// boxes with the 128-byte swizzle; rows past N read as zero.
+int make_tile_map(CUtensorMap* m, const void* base, int B, int H, int N, int d, const fa_strides& s,
+                  int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)s.n * 2u, (cuuint64_t)s.h * 2u, (cuuint64_t)s.b * 2u};
-  cuuint32_t box[4] = {64u, 128u, 1u, 1u};
+  cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
   cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -124,7 +125,7 @@ uint32_t keep_threshold(float p) {
 template <int D, bool CAUSAL, bool DROPOUT, int MODE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                cudaStream_t st) {
-  using L = fa::FwdLayout<D>;
+  using L = fa::FwdLayout<D, fa::fwd_bn<D, MODE>()>;
   constexpr bool SPLIT = MODE == fa::kFwdSplit;
   auto kern = fa::fwd_kernel<D, CAUSAL, DROPOUT, MODE>;
   const int smem = (int)(MODE == fa::kFwdSparse ? L::kSmemSparse : L::kSmem);
@@ -330,9 +331,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
     if (!aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
   }
   CUtensorMap mq, mk, mv;
+  // K/V boxes follow the kernel's key tile (64 rows for the plain d = 64 forward)
+  const int kv_rows = (!bmask && num_splits <= 1) ? (d == 64 ? fa::fwd_bn<64, fa::kFwdPlain>()
+                                                             : fa::fwd_bn<128, fa::kFwdPlain>())
+                                                  : 128;
   if ((rc = make_tile_map(&mq, q, B, H, N, d, strides[0])) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mk, k, B, H, N, d, strides[1])) != FA_OK) return rc;
-  if ((rc = make_tile_map(&mv, v, B, H, N, d, strides[2])) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mk, k, B, H, N, d, strides[1], kv_rows)) != FA_OK) return rc;
+  if ((rc = make_tile_map(&mv, v, B, H, N, d, strides[2], kv_rows)) != FA_OK) return rc;
   fa::FwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.kv_hi = kAllTiles;

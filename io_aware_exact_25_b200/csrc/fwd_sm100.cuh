@@ -94,38 +94,55 @@ enum FwdMode : int { kFwdPlain = 0, kFwdSplit = 1, kFwdSparse = 2, kFwdVarlen = 
 // FMA pipe (polynomial) and the rest on the MUFU unit, balancing the two.
 constexpr int kPolyPairsOf8 = 0;
 
-template <int D>
+// Key tile width: 64 keys for the plain forward at d = 64, 128 otherwise.
+// With 64-key tiles a CTA needs 256 TMEM columns and 96 KB of shared memory,
+// so two CTAs share an SM and each SMSP runs four softmax warps instead of two
+// (at d = 64 the softmax, not the tensor core, bounds the forward).
+template <int D, int MODE>
+__host__ __device__ constexpr int fwd_bn() { return (D == 64 && MODE == kFwdPlain) ? 64 : 128; }
+
+template <int D, int BN = 128>
 struct FwdLayout {
   // 12 warps: softmax warpgroups 0-1, and warpgroup 2 (MMA issue, TMA
   // producer, two idle warps) so that every warpgroup is whole for the
-  // register reallocation.  Launched at 168 registers a thread (3 warps per
-  // SMSP x 168 fill its 16K registers), then 200 for the softmax warpgroups
-  // and 96 for warpgroup 2: 256 * 200 + 128 * 96 = 63488 <= 384 * 168.  (At
-  // 168 for every warp the softmax spilled 48-76 bytes a thread; measured:
-  // the forward 2.8 % faster at d = 128, 7.8 % at d = 64.)
+  // register reallocation.  One CTA per SM (128-key tiles): launched at 168
+  // registers a thread (3 warps per SMSP x 168 fill its 16K registers), then
+  // 200 for the softmax warpgroups and 96 for warpgroup 2: 256 * 200 + 128 *
+  // 96 = 63488 <= 384 * 168.  (At 168 for every warp the softmax spilled
+  // 48-76 bytes a thread; measured: the forward 2.8 % faster at d = 128, 7.8 %
+  // at d = 64.)  Two CTAs per SM (64-key tiles): launched at 80, then 96 for
+  // the softmax and 48 for warpgroup 2: 256 * 96 + 128 * 48 = 30720 = 384 * 80.
+  static constexpr int kCtasPerSm = BN == 64 ? 2 : 1;
   static constexpr int kThreads = 384;
-  static constexpr uint32_t kRegsSoftmax = 200, kRegsCtl = 96;
-  static_assert(256 * kRegsSoftmax + 128 * kRegsCtl <= 384 * 168, "register split");
-  static constexpr uint32_t kHalf = 128u * 128u;     // one 128-row x 64-column bf16 half tile
-  static constexpr uint32_t kTile = 128u * D * 2u;   // one 128 x D bf16 tile
-  static constexpr int kStages = D == 128 ? 4 : 8;   // K/V ring depth
+  static constexpr uint32_t kRegsLaunch = BN == 64 ? 80 : 168;
+  static constexpr uint32_t kRegsSoftmax = BN == 64 ? 96 : 200, kRegsCtl = BN == 64 ? 48 : 96;
+  static_assert(256 * kRegsSoftmax + 128 * kRegsCtl <= 384 * kRegsLaunch, "register split");
+  static constexpr uint32_t kHalf = 128u * 128u;     // one 128-row x 64-column bf16 half tile (Q)
+  static constexpr uint32_t kHalfKV = BN * 128u;     // one BN-row x 64-column bf16 half tile (K, V)
+  static constexpr uint32_t kTile = 128u * D * 2u;   // one 128 x D bf16 tile (Q)
+  static constexpr uint32_t kTileKV = BN * D * 2u;   // one BN x D bf16 tile (K, V)
+  static constexpr int kStages = (BN == 64 || D == 64) ? 8 : 4;  // K/V ring depth
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + 2 * kTile;
-  static constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
+  static constexpr uint32_t kOffBar = kOffKV + kStages * kTileKV;
   static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t kSmem = kOffBar + kNumBars * 8 + 16;
   // block-sparse: two key-tile bit sets and three counts after the barriers
   static constexpr uint32_t kOffBits = (kSmem + 15u) & ~15u;
   static constexpr uint32_t kSmemSparse = kOffBits + 2u * kSparseWords * 4u + 16u;
-  static constexpr uint32_t kColO = 256;  // O_t at kColO + D * t
+  static constexpr uint32_t kTmemCols = 4u * BN;  // S_0, S_1 (BN columns each), O_0, O_1 (D <= BN each)
+  static constexpr uint32_t kColO = 2u * BN;      // O_t at kColO + D * t
+  static_assert(D <= BN, "O_t fits in BN columns");
   static_assert(kSmemSparse <= 232448, "shared memory budget");
+  static_assert(BN == 128 || kCtasPerSm * (kSmem + 1024) <= 233472, "two CTAs per SM");
 };
 
 template <int D, bool CAUSAL, bool DROPOUT, int MODE>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(384, (fwd_bn<D, MODE>() == 64) ? 2 : 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
-  using L = FwdLayout<D>;
+  constexpr int BN = fwd_bn<D, MODE>();  // keys per K/V tile
+  using L = FwdLayout<D, BN>;
   constexpr bool SPLIT = MODE == kFwdSplit;
   constexpr bool SPARSE = MODE == kFwdSparse;
   constexpr bool VARLEN = MODE == kFwdVarlen;
@@ -171,7 +188,7 @@ __global__ void __launch_bounds__(384, 1)
     lse_base = (long long)hh * a.total_tokens + row0;
     if (cta_tile * 256 >= seq_len) return;  // only padding (or nothing) here: no work
   }
-  const int n_kv_all = (seq_len + 127) >> 7;
+  const int n_kv_all = (seq_len + BN - 1) / BN;
   const int qt0 = 2 * cta_tile;
   // buffer extents for the bounds-checking build (unused otherwise)
   const long long rows_q = VARLEN ? a.total_tokens : a.N;
@@ -182,8 +199,8 @@ __global__ void __launch_bounds__(384, 1)
   (void)rows_q, (void)rows_k, (void)o_lim, (void)lse_lim, (void)part_rows;
   const bool act1 = (qt0 + 1) * 128 < seq_len;
   // key tiles each Q tile sees: [0, end_t)
-  const int end0 = CAUSAL ? qt0 + 1 : n_kv_all;
-  const int end1 = act1 ? (CAUSAL ? qt0 + 2 : n_kv_all) : 0;
+  const int end0 = CAUSAL ? min(n_kv_all, (qt0 + 1) * (128 / BN)) : n_kv_all;
+  const int end1 = act1 ? (CAUSAL ? min(n_kv_all, (qt0 + 2) * (128 / BN)) : n_kv_all) : 0;
   const int end_max = end0 > end1 ? end0 : end1;
   // this CTA's share [j0, j0 + span) of that range; nkv_t counts the tiles
   // tile t processes here, local index jj = j - j0 drives the pipelines
@@ -223,7 +240,7 @@ __global__ void __launch_bounds__(384, 1)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
   if (SPARSE && warp == 9) {
@@ -281,12 +298,12 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTile);
+          mbar_arrive_expect_tx(&bar_kv_full[stage], L::kTileKV);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
-          (void)FA_IN(kSiteFwdTile, row0 + kt * 128 - a.kv_row_off, 1, rows_k, a.err);
+          (void)FA_IN(kSiteFwdTile, row0 + kt * BN - a.kv_row_off, 1, rows_k, a.err);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + L::kOffKV + stage * L::kTile + h * L::kHalf, m, 64 * h,
-                        row0 + kt * 128 - a.kv_row_off, hh, wc, &bar_kv_full[stage], pol_keep);
+            tma_load_4d(smem + L::kOffKV + stage * L::kTileKV + h * L::kHalfKV, m, 64 * h,
+                        row0 + kt * BN - a.kv_row_off, hh, wc, &bar_kv_full[stage], pol_keep);
           ++issued;
           if (++stage == L::kStages) {
             stage = 0;
@@ -315,7 +332,7 @@ __global__ void __launch_bounds__(384, 1)
     // gets neither product for it; its P V product for its previous tile is
     // still issued on the step after that tile.
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // S = Q K^T, both K-major
+      constexpr uint32_t kIdS = idesc_bf16(128, BN, false, false);  // S = Q K^T, both K-major
       constexpr uint32_t kIdO = idesc_bf16(128, D, false, true);     // O += P V, V is MN-major
       bool ok = nkv_max > 0 && mbar_wait(&bar_q[0], 0, ab) && (!act1 || mbar_wait(&bar_q[1], 0, ab));
       bool issued_any = false;
@@ -325,7 +342,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t sQ = sbase + L::kOffQ + t * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + 128u * t, desc_kmajor(sQ, kk, L::kHalf), desc_kmajor(sK, kk, L::kHalf), kIdS,
+          mma_ss(tmem + (uint32_t)BN * t, desc_kmajor(sQ, kk, L::kHalf), desc_kmajor(sK, kk, L::kHalfKV), kIdS,
                  kk > 0 ? 1u : 0u);
         mma_commit(&bar_s[t]);
         issued_any = true;
@@ -334,14 +351,14 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&bar_p_half[t], j & 1, ab)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO,
+        for (int kk = 0; kk < BN / 32; ++kk)
+          mma_ts(tmem + L::kColO + D * t, tmem + (uint32_t)BN * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalfKV), kIdO,
                  (j > 0 || kk > 0) ? 1u : 0u);
         if (!mbar_wait(&bar_p[t], j & 1, ab)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 4; kk < 8; ++kk)
-          mma_ts(tmem + L::kColO + D * t, tmem + 128u * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalf), kIdO, 1u);
+        for (int kk = BN / 32; kk < BN / 16; ++kk)
+          mma_ts(tmem + L::kColO + D * t, tmem + (uint32_t)BN * t + 8u * kk, desc_mnmajor(sV, kk, L::kHalfKV), kIdO, 1u);
         mma_commit(&bar_pv[t]);
         return true;
       };
@@ -374,8 +391,8 @@ __global__ void __launch_bounds__(384, 1)
             !mbar_wait(&bar_kv_full[stage_of(posK)], phase_of(posK), ab))
           break;
         tc_fence_after();
-        const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTile;
-        const uint32_t sK = sbase + L::kOffKV + stage_of(posK) * L::kTile;
+        const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTileKV;
+        const uint32_t sK = sbase + L::kOffKV + stage_of(posK) * L::kTileKV;
         const int kt = SPARSE ? walk.next() : j0 + j;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -395,7 +412,7 @@ __global__ void __launch_bounds__(384, 1)
         const int j = nkv_max - 1, posV = 2 * j + 1;
         if (mbar_wait(&bar_kv_full[stage_of(posV)], phase_of(posV), ab)) {
           tc_fence_after();
-          const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTile;
+          const uint32_t sV = sbase + L::kOffKV + stage_of(posV) * L::kTileKV;
           bool last_ok = true;
 #pragma unroll
           for (int t = 0; t < 2; ++t)
@@ -420,7 +437,7 @@ __global__ void __launch_bounds__(384, 1)
       const int nkv = t ? nkv1 : nkv0;
       const int q_row = (qt0 + t) * 128 + r;
       const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-      const uint32_t tS = tmem + lane_off + 128u * t;
+      const uint32_t tS = tmem + lane_off + (uint32_t)BN * t;
       const uint32_t tO = tmem + lane_off + L::kColO + D * t;
       const float sl2 = a.scale_log2;
       float m_used = -INFINITY;  // running maximum (base-2 units) the P values are taken against
@@ -436,34 +453,37 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         tc_fence_after();
-        uint32_t u[4][32];
+        constexpr int kG = BN / 32;  // 32-column groups of the score tile
+        uint32_t u[kG][32];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
+        for (int c4 = 0; c4 < kG; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
         tmem_ld_wait();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
-        // key 128 jg + c is visible to query 128 (qt0 + t) + r iff c < lim;
-        // only the diagonal tile (causal) or the ragged last tile masks
-        int lim = 128;
-        if (CAUSAL && jg == qt0 + t) lim = r + 1;
-        if (!CAUSAL && jg == n_kv_all - 1 && (seq_len & 127)) lim = seq_len - jg * 128;
-        if (__any_sync(0xffffffffu, lim < 128)) {
+        for (int c4 = 0; c4 < kG; ++c4) reg_fence(u[c4]);
+        // key BN jg + c is visible to query 128 (qt0 + t) + r iff c < lim;
+        // only the diagonal tile(s) (causal) or the ragged last tile mask
+        int lim = BN;
+        if (CAUSAL) lim = min(BN, (qt0 + t) * 128 + r + 1 - jg * BN);
+        if (!CAUSAL && jg == n_kv_all - 1 && (seq_len % BN)) lim = seq_len - jg * BN;
+        if (__any_sync(0xffffffffu, lim < BN)) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < BN; ++c)
             if (c >= lim) u[c >> 5][c & 31] = 0xff800000u;  // -inf
         }
-        // row maximum: four independent 3-input max chains
-        float mx4[4];
+        // row maximum: kG independent 3-input max chains
+        float mx4[kG];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) mx4[g] = __uint_as_float(u[g][0]);
+        for (int g = 0; g < kG; ++g) mx4[g] = __uint_as_float(u[g][0]);
 #pragma unroll
         for (int c = 1; c < 31; c += 2)
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
+          for (int g = 0; g < kG; ++g)
             mx4[g] = max3(mx4[g], __uint_as_float(u[g][c]), __uint_as_float(u[g][c + 1]));
 #pragma unroll
-        for (int g = 0; g < 4; ++g) mx4[g] = fmaxf(mx4[g], __uint_as_float(u[g][31]));
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        for (int g = 0; g < kG; ++g) mx4[g] = fmaxf(mx4[g], __uint_as_float(u[g][31]));
+        float mx = mx4[0];
+#pragma unroll
+        for (int g = 1; g < kG; ++g) mx = fmaxf(mx, mx4[g]);
         const float m_new = fmaxf(m_used, mx * sl2);
         if (__any_sync(0xffffffffu, m_new > m_used + 8.0f)) {
           const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
@@ -483,13 +503,13 @@ __global__ void __launch_bounds__(384, 1)
             }
             tmem_st_wait();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
+            for (int c4 = 0; c4 < kG; ++c4) tmem_ld32(tS + 32u * c4, u[c4]);
             tmem_ld_wait();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) reg_fence(u[c4]);
-            if (__any_sync(0xffffffffu, lim < 128)) {
+            for (int c4 = 0; c4 < kG; ++c4) reg_fence(u[c4]);
+            if (__any_sync(0xffffffffu, lim < BN)) {
 #pragma unroll
-              for (int c = 0; c < 128; ++c)
+              for (int c = 0; c < BN; ++c)
                 if (c >= lim) u[c >> 5][c & 31] = 0xff800000u;
             }
           }
@@ -500,9 +520,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t mul2 = f2_pack(sl2, sl2);
         const uint64_t sub2 = f2_pack(-msub, -msub);
         uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[4][16];
+        uint32_t pk[kG][16];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < BN / 2; ++c) {
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[(2 * c) >> 5][(2 * c) & 31]),
                                              __uint_as_float(u[(2 * c + 1) >> 5][(2 * c + 1) & 31])),
                                      mul2, sub2);
@@ -518,15 +538,15 @@ __global__ void __launch_bounds__(384, 1)
           sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(p0, p1));
           if (DROPOUT) {
             // keys 2c and 2c+1 of the tile: one pair hash
-            const uint32_t w = dropout_hash(rkey, (uint32_t)(jg * 64 + c));
+            const uint32_t w = dropout_hash(rkey, (uint32_t)(jg * (BN / 2) + c));
             p0 = keep_lo(w, a.drop_threshold) ? p0 * a.drop_scale : 0.f;
             p1 = keep_hi(w, a.drop_threshold) ? p1 * a.drop_scale : 0.f;
           }
           pk[c >> 4][c & 15] = pack_bf16x2(p0, p1);
-          if (c == 31) {
-            // keys 0-63 done: publish them so O += P V can start
-            tmem_st16(tS, pk[0]);
-            tmem_st16(tS + 16u, pk[1]);
+          if (c == BN / 4 - 1) {
+            // the first half of the keys done: publish it so O += P V can start
+#pragma unroll
+            for (int h = 0; h < kG / 2; ++h) tmem_st16(tS + 16u * h, pk[h]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bar_p_half[t]);
@@ -540,8 +560,8 @@ __global__ void __launch_bounds__(384, 1)
           f2_unpack(sum2[3], s6, s7);
           l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         }
-        tmem_st16(tS + 32u, pk[2]);
-        tmem_st16(tS + 48u, pk[3]);
+#pragma unroll
+        for (int h = kG / 2; h < kG; ++h) tmem_st16(tS + 16u * h, pk[h]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar_p[t]);
@@ -618,7 +638,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
