@@ -1209,13 +1209,26 @@ cudaError_t launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const 
   return cudaGetLastError();
 }
 
+// Blocks for a grid-stride kernel of 256 threads: enough for `units` of work
+// at `per_block` units a block, at most 8 per SM.
+inline unsigned small_grid(long long units, long long per_block) {
+  const long long b = (units + per_block - 1) / per_block;
+  return (unsigned)(b < 1 ? 1 : (b > 148 * 8 ? 148 * 8 : b));
+}
+
 inline cudaError_t launch_bwd_prepare(const BwdArgs& a, int d, cudaStream_t st) {
   const int BH = a.B * a.H;
   const int npad = (a.N + 127) / 128 * 128;
+  // a block's 8 warps take 8 * (32 / lanes per row) * 4 rows per pass, and
+  // 256 float4 of the accumulator
+  const long long rows = (long long)BH * npad;
+  const long long rows_per_block = 8LL * (32 / (d * 2 / 16)) * 4;
+  const long long n4 = rows * d / 4;
+  const unsigned grid = max(small_grid(rows, rows_per_block), small_grid(n4, 256));
   if (d == 64)
-    bwd_pre_kernel<64><<<148 * 8, 256, 0, st>>>(a, BH, npad);
+    bwd_pre_kernel<64><<<grid, 256, 0, st>>>(a, BH, npad);
   else
-    bwd_pre_kernel<128><<<148 * 8, 256, 0, st>>>(a, BH, npad);
+    bwd_pre_kernel<128><<<grid, 256, 0, st>>>(a, BH, npad);
   return cudaGetLastError();
 }
 
@@ -1244,12 +1257,14 @@ inline cudaError_t launch_bwd_recompute(const CUtensorMap& mq, const CUtensorMap
 }
 
 inline cudaError_t launch_bwd_finalize(const BwdArgs& a, int d, cudaStream_t st) {
+  // one thread per 8 columns of a (padded) row
+  const unsigned grid = small_grid((long long)a.B * a.H * ((a.N + 127) / 128) * 128 * (d / 8), 256);
   if (d == 64)
-    bwd_post_kernel<64><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                 a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
+    bwd_post_kernel<64><<<grid, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
+                                              a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
   else
-    bwd_post_kernel<128><<<148 * 8, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
-                                                  a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
+    bwd_post_kernel<128><<<grid, 256, 0, st>>>(a.dq_acc, a.dq, a.B * a.H, a.H, a.N, a.dq_sb, a.dq_sh, a.dq_sn,
+                                               a.scale, a.cu_seqlens, a.seqused, a.total_tokens, a.err);
   return cudaGetLastError();
 }
 
