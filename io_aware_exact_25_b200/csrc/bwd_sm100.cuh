@@ -18,9 +18,12 @@
 //  1. row pass: D_i = dO_i . O_i and lse2_i = lse_i * log2(e) per row (rows
 //     padded to a multiple of 128 get lse2 = +inf so their P is 0), and a
 //     zeroed fp32 dQ accumulator;
-//  2. the fused recompute kernel, one CTA per 128-key tile K_j, V_j of a
-//     head, looping over the 128-row query tiles i that see it (i >= j when
-//     causal).  Per step it computes, in tensor memory with keys on the lanes,
+//  2. the fused recompute kernel, whose work item is a 128-key tile K_j, V_j
+//     of a head: a persistent grid (one CTA per SM) takes items from a
+//     counter in head-grouped order (one CTA per item with dropout,
+//     variable lengths or a block mask), and each item loops over the
+//     128-row query tiles i that see it (i >= j when causal).  Per step it
+//     computes, in tensor memory with keys on the lanes,
 //     S^T = K_j Q_i^T and dP^T = V_j dO_i^T, forms P^T and dS^T in registers,
 //     accumulates dV += P^T dO_i (P^T from tensor memory) and dK += dS^T Q_i
 //     (dS from shared memory) in tensor memory, and

@@ -10,15 +10,17 @@
 // section 3.2 (logsumexp, rescaling during accumulation).
 //
 // One CTA owns 256 query rows of one head as two 128-row tiles Q0, Q1 and
-// streams 128-key tiles K_j, V_j through a shared-memory ring.  Warp roles:
+// streams BN-key tiles K_j, V_j through a shared-memory ring: BN = 128, or 64
+// for the plain forward at d = 64, where two CTAs share an SM (fwd_bn).  Warp
+// roles:
 //   warps 0-3   softmax for Q0 (one query row per thread, TMEM lanes 0-127)
 //   warps 4-7   softmax for Q1
 //   warp  8     tcgen05 MMA issue (one thread)
 //   warp  9     TMA producer (one thread)
 //   warps 10-11 idle (they complete warpgroup 2 for the register split)
-// Tensor memory (512 columns): S_t = Q_t K_j^T (fp32, 128 columns) at
-// column 128 t; P_t (bf16, 64 columns) overwrites the first half of S_t and is
-// the A operand of O_t += P_t V_j; O_t (fp32, D columns) at 256 + D t.
+// Tensor memory (4 BN columns): S_t = Q_t K_j^T (fp32, BN columns) at column
+// BN t; P_t (bf16 pairs, BN / 2 columns) overwrites the first half of S_t and
+// is the A operand of O_t += P_t V_j; O_t (fp32, D columns) at 2 BN + D t.
 // The two Q tiles ping-pong: while one tile's softmax runs, the tensor core
 // works on the other tile's MMAs.  O_t is only rescaled by its own softmax
 // warps, after S_t(j) has completed, which implies that every earlier MMA of
