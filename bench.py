@@ -752,6 +752,146 @@ def run_ours_varlen(args, w):
     return 0
 
 
+NVLINK_GBS = 770.0  # measured peer copy per direction on this machine's B200s (nominal 900)
+
+
+def run_seqpar_emulated(args, w):
+    """``--seqpar W``: the sequence-parallel path of io_aware_exact_25_b200.seqpar
+    with its W ranks played in turn on one GPU ("FlashAttention for Efficient
+    Training", section 5.3).  Rank r holds the key window key_windows(N, W,
+    causal)[r]; a step is, per rank, fa_fwd_partial over its window and
+    fa_bwd_recompute_range over it, plus the work every rank repeats on the
+    whole sequence -- fa_merge_partials, fa_bwd_prepare, fa_bwd_finalize --
+    timed once.  The ranks share one backward workspace, so the dQ
+    accumulator ends up holding the sum the NCCL all-reduce would form and
+    the outputs are the whole problem's.  Every launch is timed with CUDA
+    events; a rank's time is its own two launches plus the repeated ones.
+    The exchanges (all-gather of the pieces, all-reduce of the accumulator)
+    do not happen on one GPU: their bytes are counted and converted to a time
+    at the measured NVLink copy rate, as a model, not a measurement."""
+    import torch
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        raise SystemExit("--seqpar plays every rank on one GPU: run it without torchrun")
+    if w.lens:
+        raise SystemExit("--seqpar takes a dense workload")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from io_aware_exact_25_b200 import binding
+    from io_aware_exact_25_b200.inputs import workload_inputs
+    from io_aware_exact_25_b200.seqpar import key_windows, tile_work
+
+    W = args.seqpar
+    x = workload_inputs(w)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    # "work": the causal split that balances the ranks; "even": equal tile counts
+    windows = key_windows(N, W, w.causal and args.seqpar_split == "work")
+    q, do = x["q"].to(dev), x["do"].to(dev)
+    kw = [x["k"][:, :, a:b].contiguous().to(dev) for a, b in windows]
+    vw = [x["v"][:, :, a:b].contiguous().to(dev) for a, b in windows]
+    part_o = torch.empty((W, B, H, N, d), dtype=torch.float32, device=dev)
+    part_lse = torch.empty((W, B, H, N), dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(q)
+    dk = [torch.empty_like(t) for t in kw]
+    dv = [torch.empty_like(t) for t in vw]
+    work = torch.empty(binding.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kwargs = dict(causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed)
+
+    # (name, rank or None for the repeated work, launch)
+    launches = []
+    for r, (a, b) in enumerate(windows):
+        launches.append(("fa_fwd_partial", r, lambda r=r, a=a: binding.fwd_partial(
+            q, kw[r], vw[r], a, part_o=part_o[r], part_lse=part_lse[r], **kwargs)))
+    launches.append(("fa_merge_partials", None, lambda: binding.merge_partials(part_o, part_lse, o=o, lse=lse)))
+    launches.append(("fa_bwd_prepare", None, lambda: binding.bwd_prepare(o, do, lse, work)))
+    for r, (a, b) in enumerate(windows):
+        if b > a:
+            launches.append(("fa_bwd_recompute_range", r, lambda r=r, a=a: binding.bwd_recompute_range(
+                q, kw[r], vw[r], do, a, work, dk=dk[r], dv=dv[r], **kwargs)))
+    launches.append(("fa_bwd_finalize", None, lambda: binding.bwd_finalize(dq, work, w.scale)))
+
+    for _ in range(args.warmup):
+        for _, _, fn in launches:
+            fn()
+    torch.cuda.synchronize(dev)
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error during warm-up")
+
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for st in range(args.steps):
+        ev[st][0].record(stream)
+        for i, (_, _, fn) in enumerate(launches):
+            fn()
+            ev[st][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if binding.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device error in the timed region")
+    ms = [sum(ev[st][i].elapsed_time(ev[st][i + 1]) for st in range(args.steps)) / args.steps
+          for i in range(len(launches))]
+    step_ms = sum(ev[st][0].elapsed_time(ev[st][-1]) for st in range(args.steps)) / args.steps
+
+    # the whole problem's identities hold for the assembled outputs
+    dk_all, dv_all = torch.cat(dk, dim=2).float(), torch.cat(dv, dim=2).float()
+    ok = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
+              and torch.isfinite(dk_all).all() and torch.isfinite(dv_all).all())
+    ok = ok and bool((dk_all.sum(dim=2).abs() <= 1e-2 * dk_all.abs().sum(dim=2) + 1e-2).all())
+    if w.p_drop == 0.0:
+        sdo = do.float().sum(dim=2)
+        ok = ok and bool(((dv_all.sum(dim=2) - sdo).abs() <= 1e-2 * dv_all.abs().sum(dim=2) + 1e-2).all())
+    if not ok:
+        raise RuntimeError("the assembled outputs failed their checks")
+
+    shared_ms = sum(m for (_, r, _), m in zip(launches, ms) if r is None)
+    rank_ms = [shared_ms + sum(m for (_, rr, _), m in zip(launches, ms) if rr == r) for r in range(W)]
+    nt = (N + 127) // 128
+    tw = tile_work(nt, w.causal)
+    rank_steps = [sum(tw[a // 128:(b + 127) // 128]) for a, b in windows]
+    ff, fb = w.fwd_flops(), w.bwd_flops()
+    # per rank: receive the other ranks' pieces (fp32 O and lse), and a ring
+    # all-reduce of the fp32 dQ accumulator sends and receives 2 (W-1)/W of it
+    gather_bytes = (W - 1) * B * H * N * (d + 1) * 4
+    reduce_bytes = int(2 * (W - 1) / W * B * H * N * d * 4)
+    model_ms = (gather_bytes + reduce_bytes) / (NVLINK_GBS * 1e9) * 1e3
+    peaks, peak_kind = load_peaks()
+    by_name = {}
+    for (name, _, _), m in zip(launches, ms):
+        by_name[name] = by_name.get(name, 0.0) + m
+    line = {
+        "metric": METRIC, "value": (ff + fb) / (step_ms * 1e-3) / 1e12, "unit": "TFLOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w), parallelism=f"sequence parallel over {W} key windows, the ranks "
+                                                       f"played in turn on one GPU"),
+        "seqpar": {
+            "world": W, "split": args.seqpar_split, "windows": windows, "rank_work_steps": rank_steps,
+            "rank_ms": rank_ms, "max_rank_ms": max(rank_ms), "mean_rank_ms": sum(rank_ms) / W,
+            "balance_max_over_mean": max(rank_ms) / (sum(rank_ms) / W),
+            "repeated_per_rank_ms": shared_ms, "launch_ms_by_entry_point": by_name,
+            "rank_compute_tflops": (ff + fb) / (max(rank_ms) * 1e-3) / 1e12,
+            "rank_compute_note": "whole-problem FLOPs over the slowest rank's kernel time: what W GPUs would "
+                                 "reach if the exchanges were free (a projection from one GPU)",
+            "exchange_bytes_per_rank": {"all_gather_received": gather_bytes, "all_reduce_ring": reduce_bytes},
+            "exchange_model_ms": model_ms,
+            "exchange_model_note": f"bytes / {NVLINK_GBS:g} GB/s measured NVLink peer copy; not measured here "
+                                   f"(one GPU)"},
+        "e2e": None, "cpu_baseline": None,
+        "gpu_launches": args.steps * len(launches),
+        "peaks": f"{peak_kind} MEASURED_PEAKS.json",
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -768,6 +908,10 @@ def main():
     ap.add_argument("--block-mask", default=None,
                     help="block-sparse run with this synthetic block mask, e.g. 'local:4,global:2' or "
                          "'random:0.25' (io_aware_exact_25_b200.inputs.block_mask)")
+    ap.add_argument("--seqpar", type=int, default=0,
+                    help="time the sequence-parallel path of this many ranks, played in turn on one GPU")
+    ap.add_argument("--seqpar-split", choices=["work", "even"], default="work",
+                    help="--seqpar key windows: balanced by causal work, or equal tile counts")
     ap.add_argument("--nvtx", action="store_true",
                     help="wrap each stage launch of the timed region in an NVTX range (for profiler timelines)")
     ap.add_argument("--no-extras", action="store_true",
@@ -785,6 +929,10 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.seqpar:
+        if args.seqpar < 1 or args.block_mask or args.splitkv:
+            ap.error("--seqpar takes a rank count >= 1 and no other forward variant")
+        return run_seqpar_emulated(args, w)
     if w.lens:
         return run_ours_varlen(args, w)
     return run_ours(args, w)

@@ -34,17 +34,43 @@ import torch.distributed as dist
 TILE = 128
 
 
-def key_windows(N: int, world: int) -> list:
-    """Key windows [(begin, end)] of the ranks: the ceil(N / 128) key tiles
-    split as evenly as possible, in rank order (a rank may get none)."""
+def tile_work(nt: int, causal: bool) -> list:
+    """Work of each of the nt key tiles in query-tile x key-tile steps: every
+    query tile sees every key tile, or, under the causal mask, key tile t is
+    seen by the query tiles t..nt-1 only (the first keys by every query)."""
+    return [nt - t for t in range(nt)] if causal else [nt] * nt
+
+
+def key_windows(N: int, world: int, causal: bool = False) -> list:
+    """Key windows [(begin, end)] of the ranks, whole 128-key tiles in rank
+    order (a rank may get none).
+
+    Without the mask the ceil(N / 128) tiles are split as evenly as
+    possible.  With it the split balances the work (``tile_work``) instead of
+    the tile count: boundary r is the tile boundary whose work prefix lies
+    closest to r/world of the total, so the early windows, which every query
+    sees, are the short ones (two ranks over 64 tiles: 19 and 45 tiles, 1045
+    and 1035 steps, where an even tile split gives 1552 and 528)."""
     if world < 1 or N < 0:
         raise ValueError("bad world size or length")
     nt = (N + TILE - 1) // TILE
-    out = []
-    for r in range(world):
-        t0, t1 = r * nt // world, (r + 1) * nt // world
-        out.append((min(t0 * TILE, N), min(t1 * TILE, N)))
-    return out
+    if not causal:
+        bounds = [r * nt // world for r in range(world + 1)]
+    else:
+        prefix = [0]
+        for wt in tile_work(nt, True):
+            prefix.append(prefix[-1] + wt)
+        bounds = [0]
+        for r in range(1, world):
+            target = r * prefix[-1] / world
+            t = bounds[-1]
+            # inner boundaries stay below the last tile, so the last rank keeps
+            # it and an empty window starts on a tile inside the sequence
+            while t < nt - 1 and abs(prefix[t + 1] - target) < abs(prefix[t] - target):
+                t += 1
+            bounds.append(t)
+        bounds.append(nt)
+    return [(min(a * TILE, N), min(b * TILE, N)) for a, b in zip(bounds, bounds[1:])]
 
 
 class CudaOps:

@@ -22,16 +22,45 @@ from io_aware_exact_25_b200.seqpar import key_windows
 
 
 def test_key_windows_tile_the_sequence():
-    for N in (1, 127, 128, 129, 1000, 4096):
+    for N in (0, 1, 127, 128, 129, 1000, 4096, 8192):
         for world in (1, 2, 3, 8, 40):
-            w = key_windows(N, world)
-            assert len(w) == world and w[0][0] == 0 and w[-1][1] == N
-            for (a, b), (c, e) in zip(w, w[1:]):
-                assert b == c and a <= b
-            for a, b in w:
-                assert a % 128 == 0 and (b == N or b % 128 == 0)
+            for causal in (False, True):
+                w = key_windows(N, world, causal)
+                assert len(w) == world and w[0][0] == 0 and w[-1][1] == N
+                for (a, b), (c, e) in zip(w, w[1:]):
+                    assert b == c and a <= b
+                for a, b in w:
+                    assert a % 128 == 0 and (b == N or b % 128 == 0)
     with pytest.raises(ValueError):
         key_windows(10, 0)
+
+
+def _steps(N, a, b, causal):
+    """Query-tile x key-tile steps of the window [a, b) by brute force: the
+    pairs (query tile i, key tile t) of which some query sees some key."""
+    nt = (N + 127) // 128
+    return sum(1 for t in range(a // 128, (b + 127) // 128) for i in range(nt) if not causal or i >= t)
+
+
+def test_causal_windows_balance_the_work():
+    """Under the causal mask no contiguous tile split has a smaller largest
+    window (brute force over every split for small cases), and the long8k
+    split at 2, 4 and 8 ranks stays within a few percent of even."""
+    import itertools
+    for nt in (1, 2, 5, 9, 16):
+        N = nt * 128
+        for world in (2, 3, 4):
+            got = max(_steps(N, a, b, True) for a, b in key_windows(N, world, True))
+            best = min(max(_steps(N, 128 * x, 128 * y, True) for x, y in zip((0,) + c, c + (nt,)))
+                       for c in itertools.combinations_with_replacement(range(nt + 1), world - 1))
+            # closest-prefix boundaries are within one tile's work of the best split
+            assert got <= best + nt, (nt, world, got, best)
+    total = _steps(8192, 0, 8192, True)
+    for world, slack in ((2, 1.01), (4, 1.04), (8, 1.12)):
+        per = [_steps(8192, a, b, True) for a, b in key_windows(8192, world, True)]
+        assert sum(per) == total and max(per) <= slack * total / world, (world, per)
+    # the even tile split it replaces: 1552 and 528 steps at two ranks
+    assert [_steps(8192, a, b, True) for a, b in key_windows(8192, 2)] == [1552, 528]
 
 
 class CpuOps:
@@ -103,7 +132,7 @@ def _worker(rank, world, out_dir, case):
         x = make_inputs(B, H, N, d, seed=61)
         keep = torch.from_numpy(oracle.dropout_mask(B, H, N, p, seed).astype(np.float64)).view(B, H, N, N)
         ops = CpuOps(keep)
-        kb, ke = seqpar.key_windows(N, world)[rank]
+        kb, ke = seqpar.key_windows(N, world, causal)[rank]
         k, v = x["k"][:, :, kb:ke], x["v"][:, :, kb:ke]
         scale = 0.3
         o, lse = seqpar.forward(x["q"], k, v, kb, causal=causal, scale=scale, dropout_p=p, seed=seed, ops=ops)

@@ -60,7 +60,7 @@ def test_windows_reproduce_the_whole_problem(cuda_device, N, d, causal, world, p
     x = make_inputs(B, H, N, d, seed=N + world)
     xd = {n: t.to(cuda_device) for n, t in x.items()}
     scale = 1.0 / math.sqrt(d)
-    o, lse, dq, dk, dv = _emulate(xd, key_windows(N, world), causal, scale, p, seed)
+    o, lse, dq, dk, dv = _emulate(xd, key_windows(N, world, causal), causal, scale, p, seed)
     kw = dict(causal=causal, p_drop=p, seed=seed)
     ro, rlse = oracle.forward(x["q"], x["k"], x["v"], scale, **kw)
     rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], scale, **kw)
