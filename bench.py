@@ -759,16 +759,19 @@ def run_seqpar_emulated(args, w):
     """``--seqpar W``: the sequence-parallel path of io_aware_exact_25_b200.seqpar
     with its W ranks played in turn on one GPU ("FlashAttention for Efficient
     Training", section 5.3).  Rank r holds the key window key_windows(N, W,
-    causal)[r]; a step is, per rank, fa_fwd_partial over its window and
+    causal)[r]; a step is, per rank, fa_fwd_partial over its window (and, with
+    the summed exchange, fa_weight_partial on its piece) and
     fa_bwd_recompute_range over it, plus the work every rank repeats on the
-    whole sequence -- fa_merge_partials, fa_bwd_prepare, fa_bwd_finalize --
-    timed once.  The ranks share one backward workspace, so the dQ
-    accumulator ends up holding the sum the NCCL all-reduce would form and
-    the outputs are the whole problem's.  Every launch is timed with CUDA
-    events; a rank's time is its own two launches plus the repeated ones.
-    The exchanges (all-gather of the pieces, all-reduce of the accumulator)
-    do not happen on one GPU: their bytes are counted and converted to a time
-    at the measured NVLink copy rate, as a model, not a measurement."""
+    whole sequence -- fa_merge_partials (of all pieces, or the one-piece
+    conversion of the sum), fa_bwd_prepare, fa_bwd_finalize -- timed once.
+    The ranks share one backward workspace, so the dQ accumulator ends up
+    holding the sum the NCCL all-reduce would form, and a torch sum of the
+    weighted pieces stands in for the forward's all-reduce: the outputs are
+    the whole problem's.  Every launch is timed with CUDA events; a rank's
+    time is its own launches plus the repeated ones.  The exchanges do not
+    happen on one GPU: their bytes are counted and converted to a time at
+    the measured NVLink copy rate, as a model, not a measurement (the stand-in
+    sum's own time is reported beside it and counted in no rank)."""
     import torch
 
     ws, rank, local = dist_env()
@@ -801,12 +804,25 @@ def run_seqpar_emulated(args, w):
     stream = torch.cuda.current_stream(dev)
     kwargs = dict(causal=w.causal, scale=w.scale, dropout_p=w.p_drop, seed=w.seed)
 
-    # (name, rank or None for the repeated work, launch)
+    # (name, rank / None for the work every rank repeats / "exchange", launch)
     launches = []
     for r, (a, b) in enumerate(windows):
         launches.append(("fa_fwd_partial", r, lambda r=r, a=a: binding.fwd_partial(
             q, kw[r], vw[r], a, part_o=part_o[r], part_lse=part_lse[r], **kwargs)))
-    launches.append(("fa_merge_partials", None, lambda: binding.merge_partials(part_o, part_lse, o=o, lse=lse)))
+    if args.seqpar_exchange == "sum":
+        # part_lse stacked is what the lse all-gather delivers; the torch sum
+        # stands in for the all-reduce of the weighted pieces (not a rank's
+        # kernel time: the exchange)
+        lse_w = torch.empty_like(lse)
+        o_sum = torch.empty((B, H, N, d), dtype=torch.float32, device=dev)
+        for r in range(W):
+            launches.append(("fa_weight_partial", r, lambda r=r: binding.weight_partial(
+                part_o[r], part_lse, r, lse=lse_w)))
+        launches.append(("all-reduce stand-in", "exchange", lambda: torch.sum(part_o, dim=0, out=o_sum)))
+        launches.append(("fa_merge_partials", None, lambda: binding.merge_partials(
+            o_sum.unsqueeze(0), lse_w.unsqueeze(0), o=o, lse=lse)))
+    else:
+        launches.append(("fa_merge_partials", None, lambda: binding.merge_partials(part_o, part_lse, o=o, lse=lse)))
     launches.append(("fa_bwd_prepare", None, lambda: binding.bwd_prepare(o, do, lse, work)))
     for r, (a, b) in enumerate(windows):
         if b > a:
@@ -851,16 +867,23 @@ def run_seqpar_emulated(args, w):
         raise RuntimeError("the assembled outputs failed their checks")
 
     shared_ms = sum(m for (_, r, _), m in zip(launches, ms) if r is None)
+    stand_in_ms = sum(m for (_, r, _), m in zip(launches, ms) if r == "exchange")
     rank_ms = [shared_ms + sum(m for (_, rr, _), m in zip(launches, ms) if rr == r) for r in range(W)]
     nt = (N + 127) // 128
     tw = tile_work(nt, w.causal)
     rank_steps = [sum(tw[a // 128:(b + 127) // 128]) for a, b in windows]
     ff, fb = w.fwd_flops(), w.bwd_flops()
-    # per rank: receive the other ranks' pieces (fp32 O and lse), and a ring
-    # all-reduce of the fp32 dQ accumulator sends and receives 2 (W-1)/W of it
-    gather_bytes = (W - 1) * B * H * N * (d + 1) * 4
-    reduce_bytes = int(2 * (W - 1) / W * B * H * N * d * 4)
-    model_ms = (gather_bytes + reduce_bytes) / (NVLINK_GBS * 1e9) * 1e3
+    # per rank, received: the forward's other pieces (fp32 O and lse) for the
+    # gather, or their lse plus a ring all-reduce of the fp32 weighted piece
+    # (2 (W-1)/W of it) for the sum; the backward's ring all-reduce of the
+    # fp32 dQ accumulator
+    ring = 2 * (W - 1) / W
+    if args.seqpar_exchange == "sum":
+        fwd_bytes = int((W - 1) * B * H * N * 4 + ring * B * H * N * d * 4)
+    else:
+        fwd_bytes = (W - 1) * B * H * N * (d + 1) * 4
+    bwd_bytes = int(ring * B * H * N * d * 4)
+    model_ms = (fwd_bytes + bwd_bytes) / (NVLINK_GBS * 1e9) * 1e3
     peaks, peak_kind = load_peaks()
     by_name = {}
     for (name, _, _), m in zip(launches, ms):
@@ -872,19 +895,21 @@ def run_seqpar_emulated(args, w):
         "config": dict(workload_config(w), parallelism=f"sequence parallel over {W} key windows, the ranks "
                                                        f"played in turn on one GPU"),
         "seqpar": {
-            "world": W, "split": args.seqpar_split, "windows": windows, "rank_work_steps": rank_steps,
+            "world": W, "split": args.seqpar_split, "exchange": args.seqpar_exchange, "windows": windows,
+            "rank_work_steps": rank_steps,
             "rank_ms": rank_ms, "max_rank_ms": max(rank_ms), "mean_rank_ms": sum(rank_ms) / W,
             "balance_max_over_mean": max(rank_ms) / (sum(rank_ms) / W),
             "repeated_per_rank_ms": shared_ms, "launch_ms_by_entry_point": by_name,
             "rank_compute_tflops": (ff + fb) / (max(rank_ms) * 1e-3) / 1e12,
             "rank_compute_note": "whole-problem FLOPs over the slowest rank's kernel time: what W GPUs would "
                                  "reach if the exchanges were free (a projection from one GPU)",
-            "exchange_bytes_per_rank": {"all_gather_received": gather_bytes, "all_reduce_ring": reduce_bytes},
+            "exchange_bytes_per_rank": {"forward": fwd_bytes, "backward_dq_all_reduce": bwd_bytes},
+            "all_reduce_stand_in_ms": stand_in_ms,
             "exchange_model_ms": model_ms,
             "exchange_model_note": f"bytes / {NVLINK_GBS:g} GB/s measured NVLink peer copy; not measured here "
                                    f"(one GPU)"},
         "e2e": None, "cpu_baseline": None,
-        "gpu_launches": args.steps * len(launches),
+        "gpu_launches": args.steps * sum(1 for _, r, _ in launches if r != "exchange"),
         "peaks": f"{peak_kind} MEASURED_PEAKS.json",
         "clocks": clocks,
     }
@@ -912,6 +937,8 @@ def main():
                     help="time the sequence-parallel path of this many ranks, played in turn on one GPU")
     ap.add_argument("--seqpar-split", choices=["work", "even"], default="work",
                     help="--seqpar key windows: balanced by causal work, or equal tile counts")
+    ap.add_argument("--seqpar-exchange", choices=["sum", "gather"], default="sum",
+                    help="--seqpar forward exchange: weighted pieces summed, or whole pieces gathered and merged")
     ap.add_argument("--nvtx", action="store_true",
                     help="wrap each stage launch of the timed region in an NVTX range (for profiler timelines)")
     ap.add_argument("--no-extras", action="store_true",

@@ -302,6 +302,20 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
  * fa_merge_partials: o bf16 [B, H, N, d] and lse [B, H, N] from num_parts
  *   pieces stacked as part_o [num_parts][B, H, N, d], part_lse
  *   [num_parts][B, H, N]: lse = ln sum_s e^lse_s, O = sum_s e^(lse_s - lse) O_s.
+ *   Every row needs a finite lse_s in some piece (a row whose pieces are all
+ *   -inf, which no query of a whole sequence has, gives undefined values).
+ * fa_weight_partial: the exchange by summation.  part_o fp32 [B, H, N, d]
+ *   is piece number `part` of num_parts (from fa_fwd_partial) and all_lse
+ *   fp32 [num_parts][B, H, N] every piece's logsumexp (an all-gather of
+ *   part_lse).  Rescales part_o in place to e^(lse_part - lse) O_part, with
+ *   lse = ln sum_s e^lse_s written to `lse` (fp32 [B, H, N]; may be null);
+ *   a row whose pieces are all -inf gets 0 and lse -inf.  The sum of the
+ *   weighted pieces over the parts (an all-reduce) is O in fp32;
+ *   fa_merge_partials with num_parts = 1 on that sum and lse converts it to
+ *   bf16.  part_o 16-byte aligned, all_lse and lse 4-byte aligned
+ *   (FA_ERR_ALIGNMENT); 1 <= num_parts <= 4096 and 0 <= part < num_parts
+ *   (FA_ERR_INVALID_ARG); a failed launch returns FA_ERR_CUDA without
+ *   updating fa_last_cuda_error (cudaGetLastError has the code).
  * fa_bwd_recompute_range: the recompute stage of fa_bwd for the window's
  *   keys: writes dk, dv of those keys (complete) and adds their part of dQ
  *   into the workspace's fp32 accumulator.  Run fa_bwd_prepare (on the full
@@ -315,6 +329,8 @@ int fa_fwd_partial(const void* q, const void* k, const void* v, float* part_o, f
                    void* stream);
 int fa_merge_partials(const float* part_o, const float* part_lse, int num_parts, void* o, float* lse, int B, int H,
                       int N, int d, void* stream);
+int fa_weight_partial(float* part_o, const float* all_lse, int num_parts, int part, float* lse, int B, int H, int N,
+                      int d, void* stream);
 size_t fa_bwd_dq_accumulator_bytes(int B, int H, int N, int d);
 int fa_bwd_recompute_range(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
                            int H, int N, int d, float scale, int causal, float dropout_p, uint64_t seed, int kv_begin,

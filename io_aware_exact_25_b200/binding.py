@@ -35,7 +35,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_splitkv", "fa_fwd_splitkv_workspa
            "fa_bwd_recompute_blocksparse", "fa_debug_fwd_timeout", "fa_debug_exp2_poly",
            "fa_debug_build", "fa_debug_bounds_record",
            "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
-           "fa_fwd_partial", "fa_merge_partials", "fa_bwd_dq_accumulator_bytes", "fa_bwd_recompute_range",
+           "fa_fwd_partial", "fa_merge_partials", "fa_weight_partial", "fa_bwd_dq_accumulator_bytes", "fa_bwd_recompute_range",
            "fa_dropout_mask", "fa_strerror",
            "fa_last_cuda_error", "fa_get_device_error", "fa_version")
 
@@ -131,6 +131,7 @@ def _open(path: str) -> ctypes.CDLL:
     lib.fa_bwd_varlen_workspace_size.restype = SZ
     lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp]
     lib.fa_merge_partials.argtypes = [vp, vp, I, vp, vp, I, I, I, I, vp]
+    lib.fa_weight_partial.argtypes = [vp, vp, I, I, vp, I, I, I, I, vp]
     lib.fa_bwd_dq_accumulator_bytes.argtypes = [I, I, I, I]
     lib.fa_bwd_dq_accumulator_bytes.restype = SZ
     lib.fa_bwd_recompute_range.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, F, I, F, U64, I, I, vp, SZ, vp]
@@ -141,7 +142,7 @@ def _open(path: str) -> ctypes.CDLL:
                lib.fa_bwd_prepare, lib.fa_bwd_recompute, lib.fa_bwd_finalize, lib.fa_bwd_noalloc,
                lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse, lib.fa_bwd_recompute_blocksparse,
                lib.fa_debug_fwd_timeout, lib.fa_debug_exp2_poly, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_fwd_partial,
-               lib.fa_merge_partials, lib.fa_bwd_recompute_range,
+               lib.fa_merge_partials, lib.fa_weight_partial, lib.fa_bwd_recompute_range,
                lib.fa_dropout_mask, lib.fa_get_device_error,
                lib.fa_last_cuda_error, lib.fa_version, lib.fa_debug_build, lib.fa_debug_bounds_record):
         fn.restype = I
@@ -463,6 +464,23 @@ def merge_partials(part_o, part_lse, o=None, lse=None, stream=None):
     rc = load().fa_merge_partials(_ptr(part_o), _ptr(part_lse), S, _ptr(o), _ptr(lse), B, H, N, d, _stream(stream))
     _call(rc, "fa_merge_partials")
     return o, lse
+
+
+def weight_partial(part_o, all_lse, part, lse=None, stream=None):
+    """``fa_weight_partial``: rescale the piece part_o (fp32 [B,H,N,d], in
+    place) to e^(lse_part - lse) O_part given every piece's logsumexp all_lse
+    (fp32 [S,B,H,N]); returns (part_o, lse) with lse = ln sum_s e^lse_s."""
+    S = all_lse.shape[0]
+    B, H, N, d = part_o.shape
+    if part_o.dtype != torch.float32 or all_lse.dtype != torch.float32:
+        raise ValueError("pieces are fp32")
+    if not (part_o.is_contiguous() and all_lse.is_contiguous()) or tuple(all_lse.shape) != (S, B, H, N):
+        raise ValueError("part_o must be dense [B,H,N,d] and all_lse dense [S,B,H,N]")
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=part_o.device)
+    rc = load().fa_weight_partial(_ptr(part_o), _ptr(all_lse), S, int(part), _ptr(lse), B, H, N, d, _stream(stream))
+    _call(rc, "fa_weight_partial")
+    return part_o, lse
 
 
 def dq_accumulator_bytes(B, H, N, d) -> int:

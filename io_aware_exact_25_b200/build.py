@@ -10,7 +10,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfa_sm100.so")
 DEBUG_LIB = os.path.join(PKG, "libfa_sm100_debug.so")
-SOURCES = [os.path.join(PKG, "csrc", "fa_api.cu"), os.path.join(PKG, "csrc", "fa_noalloc.cu")]
+SOURCES = [os.path.join(PKG, "csrc", n) for n in ("fa_api.cu", "fa_noalloc.cu", "fa_seqpar.cu")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-shared"]
 

@@ -13,9 +13,17 @@ key rows [kv_begin, kv_begin + Nk)), the windows of the ranks tiling the
 sequence in rank order (``key_windows``).
 
   forward:  each rank computes the softmax piece of every query over its
-            keys (``fa_fwd_partial``: O_r normalised over its keys, lse_r);
-            the pieces are all-gathered (NCCL) and every rank merges them
-            (``fa_merge_partials``) into the full O and lse.
+            keys (``fa_fwd_partial``: O_r normalised over its keys, lse_r).
+            By default the pieces meet in a sum: the lse_r are all-gathered
+            (NCCL), every rank rescales its own piece to
+            e^(lse_r - lse) O_r (``fa_weight_partial``), one all-reduce adds
+            the weighted pieces into O in fp32 and a one-piece
+            ``fa_merge_partials`` converts it to bf16.  With
+            ``exchange="gather"`` the whole pieces are all-gathered instead
+            and every rank merges all of them; per rank that receives
+            (W - 1) B H N (d + 1) fp32 values against the sum's
+            2 (W - 1) / W B H N d (ring all-reduce) plus the lse gather --
+            the same at two ranks, a quarter at eight.
   backward: each rank forms D = dO . O and the scaled lse from the full O
             (``fa_bwd_prepare``), recomputes its key window
             (``fa_bwd_recompute_range``: its dK, dV complete, its part of dQ
@@ -86,6 +94,9 @@ class CudaOps:
     def merge(self, part_o, part_lse):
         return self.b.merge_partials(part_o, part_lse)
 
+    def weight(self, part_o, all_lse, part):
+        return self.b.weight_partial(part_o, all_lse, part)
+
     def bwd_begin(self, o, do, lse):
         B, H, N, d = o.shape
         ws = torch.empty(self.b.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=o.device)
@@ -104,19 +115,29 @@ class CudaOps:
         return self.b.bwd_finalize(torch.empty_like(q), ws, scale)
 
 
-def forward(q, k, v, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, group=None, ops=None):
-    """Full O and lse on every rank from the ranks' key windows."""
+def _all_gather(t, world, group):
+    flat = torch.empty(world * t.numel(), dtype=t.dtype, device=t.device)
+    dist.all_gather_into_tensor(flat, t.contiguous().view(-1), group=group)
+    return flat.view((world,) + tuple(t.shape))
+
+
+def forward(q, k, v, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, group=None, ops=None,
+            exchange="sum"):
+    """Full O and lse on every rank from the ranks' key windows; the ranks'
+    windows follow their order in ``group``."""
+    if exchange not in ("sum", "gather"):
+        raise ValueError("exchange is 'sum' or 'gather'")
     ops = ops or CudaOps()
     d = q.shape[-1]
     scale = scale if scale is not None else d ** -0.5
     part_o, part_lse = ops.fwd_partial(q, k, v, kv_begin, causal, scale, dropout_p, seed)
     world = dist.get_world_size(group)
-    gathered = []
-    for t in (part_o, part_lse):
-        flat = torch.empty(world * t.numel(), dtype=t.dtype, device=t.device)
-        dist.all_gather_into_tensor(flat, t.contiguous().view(-1), group=group)
-        gathered.append(flat.view((world,) + tuple(t.shape)))
-    return ops.merge(*gathered)
+    if exchange == "gather":
+        return ops.merge(_all_gather(part_o, world, group), _all_gather(part_lse, world, group))
+    all_lse = _all_gather(part_lse, world, group)
+    part_o, lse = ops.weight(part_o, all_lse, dist.get_rank(group))
+    dist.all_reduce(part_o, op=dist.ReduceOp.SUM, group=group)
+    return ops.merge(part_o.unsqueeze(0), lse.unsqueeze(0))
 
 
 def backward(q, k, v, o, do, lse, kv_begin, causal=False, scale=None, dropout_p=0.0, seed=0, group=None, ops=None):

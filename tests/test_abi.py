@@ -221,3 +221,16 @@ def test_key_window_arguments_are_rejected_before_launch(lib):
     assert rng(256, 256) == binding.FA_OK  # an empty window adds nothing and launches nothing
     assert lib.fa_merge_partials(16, 16, 0, 16, 16, 1, 2, 100, 64, None) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_merge_partials(16, 18, 2, 16, 16, 1, 2, 100, 64, None) == binding.FA_ERR_ALIGNMENT
+
+
+def test_weight_partial_arguments_are_rejected_before_launch(lib):
+    def w(po=16, al=16, S=2, part=0, lse=16, d=64, B=1):
+        return lib.fa_weight_partial(po, al, S, part, lse, B, 2, 100, d, None)
+
+    for S, part in ((0, 0), (2, 2), (2, -1), (4097, 0)):
+        assert w(S=S, part=part) == binding.FA_ERR_INVALID_ARG, (S, part)
+    assert w(d=80) == binding.FA_ERR_UNSUPPORTED
+    assert w(po=None) == binding.FA_ERR_INVALID_ARG and w(al=None) == binding.FA_ERR_INVALID_ARG
+    assert w(po=24) == binding.FA_ERR_ALIGNMENT and w(al=18) == binding.FA_ERR_ALIGNMENT
+    assert w(lse=18) == binding.FA_ERR_ALIGNMENT
+    assert w(B=0) == binding.FA_OK and w(B=-1) == binding.FA_ERR_INVALID_ARG  # empty: nothing launched

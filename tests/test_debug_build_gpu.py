@@ -132,8 +132,8 @@ def test_varlen_with_padded_slots(cuda_device, d):
 
 
 def test_sequence_parallel_pieces(cuda_device):
-    """fa_fwd_partial, fa_merge_partials and fa_bwd_recompute_range over three
-    key windows, one of them ragged."""
+    """fa_fwd_partial, fa_merge_partials, fa_weight_partial and
+    fa_bwd_recompute_range over three key windows, one of them ragged."""
     B, H, N, d = 1, 2, 700, 128
     x = _dev(make_inputs(B, H, N, d, seed=21), cuda_device)
     windows = [(0, 256), (256, 512), (512, N)]
@@ -142,7 +142,9 @@ def test_sequence_parallel_pieces(cuda_device):
         parts = [binding.fwd_partial(x["q"], x["k"][:, :, a:b].contiguous(), x["v"][:, :, a:b].contiguous(), a,
                                      causal=True) for a, b in windows]
         o, lse = binding.merge_partials(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
-        out = [o, lse]
+        all_lse = torch.stack([p[1] for p in parts]).contiguous()
+        weighted = [binding.weight_partial(p[0].clone(), all_lse, r)[0] for r, p in enumerate(parts)]
+        out = [o, lse] + weighted
         for a, b in windows:
             ws = torch.empty(binding.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=cuda_device)
             binding.bwd_prepare(o, x["do"], lse, ws)
@@ -152,7 +154,7 @@ def test_sequence_parallel_pieces(cuda_device):
         return out
 
     ref, got = _run_both(run)
-    _same(ref, got, ["o", "lse"] + [f"{n}{w}" for w in range(3) for n in ("dk", "dv")])
+    _same(ref, got, ["o", "lse"] + [f"w{r}" for r in range(3)] + [f"{n}{w}" for w in range(3) for n in ("dk", "dv")])
 
 
 def test_noalloc_backward(cuda_device):

@@ -3,8 +3,9 @@ with the gloo backend, world size 2 and 3.
 
 "FlashAttention for Efficient Training", section 5.3 (Sequence Parallelism
 for Long Contexts).  The orchestration -- key windows per rank, the
-all-gather of the softmax pieces and their merge, the all-reduce of the dQ
-accumulators -- runs here unchanged; the per-rank compute steps come from a
+forward exchange (the lse all-gather and the all-reduce of the weighted
+pieces, or the all-gather of whole pieces and their merge), the all-reduce
+of the dQ accumulators -- runs here unchanged; the per-rank compute steps come from a
 CPU double written in fp64 torch from the definition (the CUDA steps are
 tested against the oracle on the GPU, tests/test_seqpar_gpu.py).  The
 ranks' results must equal the fp64 oracle run on the whole problem.
@@ -93,6 +94,12 @@ class CpuOps:
         w = torch.where(torch.isneginf(all_lse), torch.zeros_like(all_lse), torch.exp(all_lse - lse))
         return (w[..., None] * all_o).sum(0), lse
 
+    def weight(self, part_o, all_lse, part):
+        lse = torch.logsumexp(all_lse, dim=0)
+        mine = all_lse[part]
+        w = torch.where(torch.isneginf(mine), torch.zeros_like(mine), torch.exp(mine - lse))
+        return part_o * w[..., None], lse
+
     def bwd_begin(self, o, do, lse):
         return {"D": (do.double() * o.double()).sum(-1), "lse": lse.double(),
                 "acc": torch.zeros(o.shape, dtype=torch.float64)}
@@ -115,7 +122,9 @@ class CpuOps:
         return ws["acc"]
 
 
-CASES = {"causal": (True, 0.0), "noncausal_dropout": (False, 0.2)}
+# name: (causal, dropout p, forward exchange)
+CASES = {"causal": (True, 0.0, "sum"), "noncausal_dropout": (False, 0.2, "sum"),
+         "causal_gather": (True, 0.0, "gather")}
 
 
 def _worker(rank, world, out_dir, case):
@@ -127,7 +136,7 @@ def _worker(rank, world, out_dir, case):
         import oracle
         from io_aware_exact_25_b200 import seqpar
         from io_aware_exact_25_b200.inputs import make_inputs
-        causal, p = CASES[case]
+        causal, p, exchange = CASES[case]
         B, H, N, d, seed = 1, 2, 300, 16, 7
         x = make_inputs(B, H, N, d, seed=61)
         keep = torch.from_numpy(oracle.dropout_mask(B, H, N, p, seed).astype(np.float64)).view(B, H, N, N)
@@ -135,7 +144,8 @@ def _worker(rank, world, out_dir, case):
         kb, ke = seqpar.key_windows(N, world, causal)[rank]
         k, v = x["k"][:, :, kb:ke], x["v"][:, :, kb:ke]
         scale = 0.3
-        o, lse = seqpar.forward(x["q"], k, v, kb, causal=causal, scale=scale, dropout_p=p, seed=seed, ops=ops)
+        o, lse = seqpar.forward(x["q"], k, v, kb, causal=causal, scale=scale, dropout_p=p, seed=seed, ops=ops,
+                                exchange=exchange)
         dq, dk, dv = seqpar.backward(x["q"], k, v, o, x["do"], lse, kb, causal=causal, scale=scale, dropout_p=p,
                                      seed=seed, ops=ops)
         for name, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
@@ -152,7 +162,7 @@ def test_ranks_reproduce_the_whole_problem(tmp_path, world, case):
                        start_method="spawn", join=True)
     import oracle
     from io_aware_exact_25_b200.inputs import make_inputs
-    causal, p = CASES[case]
+    causal, p, _ = CASES[case]
     B, H, N, d, seed = 1, 2, 300, 16, 7
     x = make_inputs(B, H, N, d, seed=61)
     kw = dict(causal=causal, p_drop=p, seed=seed)

@@ -1,13 +1,15 @@
 """The per-rank pieces of sequence parallelism (fa_fwd_partial,
-fa_merge_partials, fa_bwd_recompute_range) against the fp64 oracle (GPU).
+fa_merge_partials, fa_weight_partial, fa_bwd_recompute_range) against the
+fp64 oracle (GPU).
 
 "FlashAttention for Efficient Training", section 5.3 (Sequence Parallelism
 for Long Contexts).  One GPU plays every rank in turn: each key window gets
-its own softmax piece and its own backward workspace; the pieces are stacked
-and merged, and the windows' fp32 dQ accumulators summed -- the data the
-NCCL all-gather and all-reduce of io_aware_exact_25_b200.seqpar exchange
-(their bookkeeping is tested over gloo in tests/test_seqpar_gloo.py).
-Every element is compared with the bar of tests/parity.py.
+its own softmax piece and its own backward workspace; the pieces are either
+stacked and merged or weighted and summed, and the windows' fp32 dQ
+accumulators summed -- the data the NCCL all-gather and all-reduce of
+io_aware_exact_25_b200.seqpar exchange (their bookkeeping is tested over
+gloo in tests/test_seqpar_gloo.py; here torch sums stand in for the
+all-reduce).  Every element is compared with the bar of tests/parity.py.
 """
 import math
 
@@ -88,3 +90,84 @@ def test_one_window_is_the_dense_path(cuda_device):
     assert (lse1 - lse0).abs().max().item() <= 1e-5
     assert torch.equal(dk1, dk0) and torch.equal(dv1, dv0)
     assert (dq1.float() - dq0.float()).abs().max().item() <= 2 ** -7
+
+
+def _weighted_forward(x, windows, causal, scale, p, seed):
+    """The summed exchange: every rank weights its own piece with all the
+    pieces' lse, the weighted pieces are added (the all-reduce) and one
+    one-piece merge converts the sum to bf16."""
+    q = x["q"]
+    parts = [binding.fwd_partial(q, x["k"][:, :, a:b].contiguous(), x["v"][:, :, a:b].contiguous(), a,
+                                 causal=causal, scale=scale, dropout_p=p, seed=seed) for a, b in windows]
+    all_lse = torch.stack([t[1] for t in parts]).contiguous()
+    lse_w = None
+    for r, (po, _) in enumerate(parts):
+        _, lse_r = binding.weight_partial(po, all_lse, r)
+        if lse_w is None:
+            lse_w = lse_r
+        else:
+            assert torch.equal(lse_r, lse_w)  # every rank forms the same lse
+    total = torch.stack([t[0] for t in parts]).sum(0)
+    o, lse = binding.merge_partials(total.unsqueeze(0).contiguous(), lse_w.unsqueeze(0).contiguous())
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    return o, lse, parts
+
+
+@pytest.mark.parametrize("N,d,causal,world,p", [
+    (1000, 128, True, 2, 0.0), (1000, 64, False, 3, 0.0), (777, 128, True, 4, 0.1), (384, 64, True, 8, 0.0),
+    (2048, 128, True, 5, 0.0)])
+def test_weighted_pieces_sum_to_the_whole_problem(cuda_device, N, d, causal, world, p):
+    B, H, seed = 1, 2, 23
+    x = make_inputs(B, H, N, d, seed=N + world)
+    xd = {n: t.to(cuda_device) for n, t in x.items()}
+    scale = 1.0 / math.sqrt(d)
+    windows = key_windows(N, world, causal)
+    o, lse, parts = _weighted_forward(xd, windows, causal, scale, p, seed)
+    ro, rlse = oracle.forward(x["q"], x["k"], x["v"], scale, causal=causal, p_drop=p, seed=seed)
+    parity.check("O", o, ro)
+    parity.check_lse(lse, rlse)
+    # against the gather exchange: the same lse, O within one bf16 rounding
+    xd2 = {n: t.to(cuda_device) for n, t in x.items()}
+    parts2 = [binding.fwd_partial(xd2["q"], xd2["k"][:, :, a:b].contiguous(), xd2["v"][:, :, a:b].contiguous(), a,
+                                  causal=causal, scale=scale, dropout_p=p, seed=seed) for a, b in windows]
+    og, lseg = binding.merge_partials(torch.stack([t[0] for t in parts2]), torch.stack([t[1] for t in parts2]))
+    torch.cuda.synchronize()
+    assert (lse - lseg).abs().max().item() <= 1e-5
+    assert ((o.float() - og.float()).abs() <= og.float().abs() * 2 ** -7 + 1e-6).all()
+
+
+@pytest.mark.parametrize("d,S", [(64, 1), (128, 3), (64, 40), (128, 33)])
+def test_weight_partial_against_its_definition(cuda_device, d, S):
+    """Random pieces and logsumexps, some -inf and one row -inf in every
+    piece, against the definition in fp64: lse = ln sum_s e^lse_s,
+    piece * e^(lse_part - lse); 0 and lse = -inf where nothing is seen.
+    S = 33 and 40 exceed the 32 lanes that share a row's reduction."""
+    B, H, N = 2, 3, 130
+    g = torch.Generator().manual_seed(d + S)
+    all_lse = torch.randn((S, B, H, N), generator=g, dtype=torch.float64) * 6
+    all_lse[torch.rand((S, B, H, N), generator=g) < 0.3] = float("-inf")
+    all_lse[:, 1, 2, 7] = float("-inf")  # a row that no piece sees
+    all_lse[:, 0, 0, 5] = 80.0  # equal pieces: lse = 80 + ln S
+    pieces = torch.randn((S, B, H, N, d), generator=g, dtype=torch.float64)
+    all_lse = all_lse.float().double()  # the values the kernel sees
+    ref_lse = torch.logsumexp(all_lse, dim=0)
+    lse_dev = all_lse.float().to(cuda_device).contiguous()
+    for part in sorted({0, S // 2, S - 1}):
+        po = pieces[part].float().to(cuda_device).contiguous()
+        out, lse = binding.weight_partial(po, lse_dev, part)
+        torch.cuda.synchronize()
+        mine = all_lse[part]
+        w = torch.where(torch.isneginf(mine), torch.zeros_like(mine), torch.exp(mine - ref_lse))
+        w = torch.nan_to_num(w, nan=0.0)
+        ref = pieces[part].float().double() * w[..., None]
+        got = out.double().cpu()
+        # fp32 arithmetic: lse rounded at |lse| <= 84 (half an ulp 3.8e-6) plus
+        # the sum of up to 40 terms and logf, exp of the difference
+        assert torch.allclose(got, ref, rtol=2e-5, atol=1e-30), (got - ref).abs().max().item()
+        assert torch.equal(got[w == 0], torch.zeros_like(got[w == 0]))
+        lc = lse.double().cpu()
+        fin = torch.isfinite(ref_lse)
+        assert torch.equal(torch.isneginf(lc), ~fin)
+        assert ((lc[fin] - ref_lse[fin]).abs() <= 1e-5 + 1e-7 * ref_lse[fin].abs()).all()
+        assert abs(lc[0, 0, 5].item() - (80 + math.log(S))) <= 1e-4
