@@ -9,10 +9,11 @@
 // of all ranks then meet in one sum (an all-reduce) instead of each rank
 // gathering and merging every piece.
 //
-// One warp per (b, h, row): the lanes reduce the num_parts logsumexps (max,
-// then the sum of exponentials), and each lane rescales d/32 of the row's
-// floats in place.  Memory-bound: the piece is read and written once (at
-// long8k, B=2 H=16 N=8192 d=128: 128 MiB each way).
+// A warp takes 32 rows: lane l reduces the num_parts logsumexps of row l
+// (max, then the sum of exponentials; no shuffles, coalesced across lanes),
+// then the warp rescales the 32 rows in place, each lane d/32 floats of a row
+// with that row's weight taken from its lane.  Memory-bound: the piece is
+// read and written once (at long8k, B=2 H=16 N=8192 d=128: 128 MiB each way).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -27,44 +28,62 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     weight_partial_kernel(float* __restrict__ part_o, const float* __restrict__ all_lse, int num_parts, int part,
                           float* __restrict__ lse_out, long long rows) {
-  constexpr int kPer = D / 32;
+  constexpr int kPer = D / 32;  // floats of a row per lane
+  constexpr int kBatch = 8;     // rows loaded before any is stored
   const int lane = threadIdx.x & 31;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long r = warp0; r < rows; r += nwarps) {
-    // the row's floats are loaded first, so their latency overlaps the
-    // reduction of the logsumexps
-    float* row = part_o + r * D + lane * kPer;
-    float v[kPer];
-    if constexpr (kPer == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(row);
-      v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
-    } else {
-      const float2 t = *reinterpret_cast<const float2*>(row);
-      v[0] = t.x, v[1] = t.y;
+  for (long long r0 = warp0 * 32; r0 < rows; r0 += nwarps * 32) {
+    // lane l reduces the logsumexps of row r0 + l (consecutive lanes read
+    // consecutive rows of each piece)
+    const long long rl = r0 + lane;
+    float w = 0.f;
+    if (rl < rows) {
+      float mx = -INFINITY;
+      for (int s = 0; s < num_parts; ++s) mx = fmaxf(mx, all_lse[(long long)s * rows + rl]);
+      float lse = -INFINITY;
+      if (mx != -INFINITY) {
+        float sum = 0.f;
+        for (int s = 0; s < num_parts; ++s) {
+          const float ls = all_lse[(long long)s * rows + rl];
+          sum += ls == -INFINITY ? 0.f : expf(ls - mx);
+        }
+        lse = mx + logf(sum);
+        const float mine = all_lse[(long long)part * rows + rl];
+        w = mine == -INFINITY ? 0.f : expf(mine - lse);
+      }
+      if (lse_out) lse_out[rl] = lse;
     }
-    float mx = -INFINITY;
-    for (int s = lane; s < num_parts; s += 32) mx = fmaxf(mx, all_lse[(long long)s * rows + r]);
+    // then the warp rescales its rows, each lane d/32 floats of every row,
+    // kBatch rows in flight at a time
+    const int nr = rows - r0 < 32 ? (int)(rows - r0) : 32;
+    for (int j0 = 0; j0 < nr; j0 += kBatch) {
+      float v[kBatch][kPer];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float w = 0.f, lse = -INFINITY;
-    if (mx != -INFINITY) {
-      float sum = 0.f;
-      for (int s = lane; s < num_parts; s += 32) {
-        const float ls = all_lse[(long long)s * rows + r];
-        sum += ls == -INFINITY ? 0.f : expf(ls - mx);
+      for (int j = 0; j < kBatch; ++j) {
+        if (j0 + j < nr) {
+          const float* row = part_o + (r0 + j0 + j) * D + lane * kPer;
+          if constexpr (kPer == 4) {
+            const float4 t = *reinterpret_cast<const float4*>(row);
+            v[j][0] = t.x, v[j][1] = t.y, v[j][2] = t.z, v[j][3] = t.w;
+          } else {
+            const float2 t = *reinterpret_cast<const float2*>(row);
+            v[j][0] = t.x, v[j][1] = t.y;
+          }
+        }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      lse = mx + logf(sum);
-      const float mine = all_lse[(long long)part * rows + r];
-      w = mine == -INFINITY ? 0.f : expf(mine - lse);
+      for (int j = 0; j < kBatch; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+        if (j0 + j < nr) {
+          float* row = part_o + (r0 + j0 + j) * D + lane * kPer;
+          if constexpr (kPer == 4)
+            *reinterpret_cast<float4*>(row) = make_float4(v[j][0] * wj, v[j][1] * wj, v[j][2] * wj, v[j][3] * wj);
+          else
+            *reinterpret_cast<float2*>(row) = make_float2(v[j][0] * wj, v[j][1] * wj);
+        }
+      }
     }
-    if constexpr (kPer == 4)
-      *reinterpret_cast<float4*>(row) = make_float4(v[0] * w, v[1] * w, v[2] * w, v[3] * w);
-    else
-      *reinterpret_cast<float2*>(row) = make_float2(v[0] * w, v[1] * w);
-    if (lse_out && lane == 0) lse_out[r] = lse;
   }
 }
 
@@ -82,7 +101,7 @@ extern "C" int fa_weight_partial(float* part_o, const float* all_lse, int num_pa
     return FA_ERR_ALIGNMENT;
   const long long rows = (long long)B * H * N;
   if (rows * num_parts > (1ll << 40)) return FA_ERR_TOO_LARGE;
-  const long long want = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const long long want = (rows + 32 * kWarpsPerBlock - 1) / (32 * kWarpsPerBlock);
   const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64)
