@@ -171,3 +171,43 @@ def test_weight_partial_against_its_definition(cuda_device, d, S):
         assert torch.equal(torch.isneginf(lc), ~fin)
         assert ((lc[fin] - ref_lse[fin]).abs() <= 1e-5 + 1e-7 * ref_lse[fin].abs()).all()
         assert abs(lc[0, 0, 5].item() - (80 + math.log(S))) <= 1e-4
+
+
+def test_one_rank_nccl_group_runs_the_cuda_orchestration(cuda_device, tmp_path):
+    """seqpar.forward / seqpar.backward with the CUDA steps and real NCCL
+    collectives over a one-rank group (no kernel waits on another rank):
+    one window holds every key, so O, lse, dK and dV are the dense path's and
+    every output meets the oracle, for both forward exchanges."""
+    import torch.distributed as dist
+    from datetime import timedelta
+    from io_aware_exact_25_b200 import seqpar
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised in this process")
+    B, H, N, d = 1, 2, 700, 128
+    x = make_inputs(B, H, N, d, seed=77)
+    xd = {n: t.to(cuda_device) for n, t in x.items()}
+    o0, lse0 = binding.fwd(xd["q"], xd["k"], xd["v"], causal=True)
+    dq0, dk0, dv0 = binding.bwd(xd["q"], xd["k"], xd["v"], o0, xd["do"], lse0, causal=True)
+    scale = 1.0 / math.sqrt(d)
+    ro, rlse = oracle.forward(x["q"], x["k"], x["v"], scale, causal=True)
+    rdq, _, _ = oracle.backward_q(x["q"], x["k"], x["v"], x["do"], scale, causal=True)
+    rdk, rdv = oracle.backward_kv(x["q"], x["k"], x["v"], x["do"], scale, causal=True)
+    dist.init_process_group("nccl", init_method="file://" + str(tmp_path / "store"), rank=0, world_size=1,
+                            timeout=timedelta(seconds=60))
+    try:
+        for exchange in ("sum", "gather"):
+            o, lse = seqpar.forward(xd["q"], xd["k"], xd["v"], 0, causal=True, exchange=exchange)
+            dq, dk, dv = seqpar.backward(xd["q"], xd["k"], xd["v"], o, xd["do"], lse, 0, causal=True)
+            torch.cuda.synchronize()
+            assert binding.device_error() == 0
+            assert (o.float() - o0.float()).abs().max().item() <= 2 ** -8, exchange
+            assert (lse - lse0).abs().max().item() <= 1e-5, exchange
+            assert torch.equal(dk, dk0) and torch.equal(dv, dv0), exchange
+            assert (dq.float() - dq0.float()).abs().max().item() <= 2 ** -7, exchange
+            parity.check("O", o, ro)
+            parity.check_lse(lse, rlse)
+            parity.check("dQ", dq, rdq)
+            parity.check("dK", dk, rdk)
+            parity.check("dV", dv, rdv)
+    finally:
+        dist.destroy_process_group()
