@@ -302,8 +302,7 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
  * fa_merge_partials: o bf16 [B, H, N, d] and lse [B, H, N] from num_parts
  *   pieces stacked as part_o [num_parts][B, H, N, d], part_lse
  *   [num_parts][B, H, N]: lse = ln sum_s e^lse_s, O = sum_s e^(lse_s - lse) O_s.
- *   Every row needs a finite lse_s in some piece (a row whose pieces are all
- *   -inf, which no query of a whole sequence has, gives undefined values).
+ *   A row whose pieces are all -inf gets O = 0 and lse = -inf.
  * fa_weight_partial: the exchange by summation.  part_o fp32 [B, H, N, d]
  *   is piece number `part` of num_parts (from fa_fwd_partial) and all_lse
  *   fp32 [num_parts][B, H, N] every piece's logsumexp (an all-gather of

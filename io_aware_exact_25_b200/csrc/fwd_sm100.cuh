@@ -644,45 +644,92 @@ __global__ void __launch_bounds__(384, (fwd_bn<D, MODE>() == 64) ? 2 : 1)
   }
 }
 
-// Merge the split-KV partials of one row: lse = ln sum_s exp(lse_s) and
+// Merge the split-KV partials: per row lse = ln sum_s exp(lse_s) and
 // O = sum_s exp(lse_s - lse) O_s, the exact combination of softmax pieces over
-// disjoint key ranges.  One warp per row.
+// disjoint key ranges; a row whose pieces are all -inf gets O = 0 and
+// lse = -inf.  A warp takes G rows at a time: lane l < G reduces the pieces'
+// logsumexps of row l (consecutive lanes read consecutive rows of each
+// piece), then the warp combines the rows four at a time, each lane d/32
+// floats of a row, so that four rows' loads of a piece are in flight
+// together.  G is the largest power of two up to 32 that still gives every
+// warp of the grid a group, so a problem of few rows (one long sequence of
+// one head) keeps the whole grid busy.  Memory-bound: every piece is read
+// once and O written once.
 template <int D>
 __global__ void __launch_bounds__(256) splitkv_combine_kernel(const FwdArgs a) {
   constexpr int kPer = D / 32;
-  const int BH = a.B * a.H;
-  const long long rows = (long long)BH * a.N;
+  constexpr int kRows = 4;
+  const int S = a.num_splits;
+  const long long rows = (long long)a.B * a.H * a.N;
   const int lane = threadIdx.x & 31;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const long long o_lim = extent4(a.B, a.H, a.N, D, a.o_sb, a.o_sh, a.o_sn);
   (void)o_lim;
-  for (long long r = warp0; r < rows; r += nwarps) {
-    if (!FA_IN(kSiteCombine, (long long)(a.num_splits - 1) * rows + r, 1, (long long)a.num_splits * rows, a.err))
-      continue;
-    float mx = -INFINITY;
-    for (int s = 0; s < a.num_splits; ++s) mx = fmaxf(mx, a.part_lse[(size_t)s * rows + r]);
-    float acc[kPer];
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-    float wsum = 0.f;
-    for (int s = 0; s < a.num_splits; ++s) {
-      const float ls = a.part_lse[(size_t)s * rows + r];
-      const float w = (ls == -INFINITY) ? 0.f : __expf(ls - mx);
-      wsum += w;
-      const float* src = a.part_o + ((size_t)s * rows + r) * D + lane * kPer;
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+  int G = 32;
+  while (G > 1 && (long long)G * nwarps > rows) G >>= 1;
+  for (long long r0 = warp0 * G; r0 < rows; r0 += nwarps * G) {
+    const long long rl = r0 + lane;
+    float mx = -INFINITY, inv = 0.f;
+    if (lane < G && rl < rows) {
+      for (int s = 0; s < S; ++s) mx = fmaxf(mx, a.part_lse[(long long)s * rows + rl]);
+      float lse = -INFINITY;
+      if (mx != -INFINITY) {
+        float wsum = 0.f;
+        for (int s = 0; s < S; ++s) {
+          const float ls = a.part_lse[(long long)s * rows + rl];
+          wsum += ls == -INFINITY ? 0.f : __expf(ls - mx);
+        }
+        inv = 1.f / wsum;
+        lse = mx + logf(wsum);
+      }
+      a.lse[rl] = lse;
     }
-    const float inv = 1.f / wsum;
-    const int bh = (int)(r / a.N), i = (int)(r - (long long)bh * a.N);
-    const int b_ = bh / a.H, h_ = bh - b_ * a.H;
-    const long long ooff = b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn;
-    if (!FA_IN(kSiteCombine, ooff, D, o_lim, a.err)) continue;
-    __nv_bfloat16* orow = a.o + ooff + lane * kPer;
+    const int nr = rows - r0 < G ? (int)(rows - r0) : G;
+    for (int j0 = 0; j0 < nr; j0 += kRows) {
+      float mxj[kRows], invj[kRows], acc[kRows][kPer];
 #pragma unroll
-    for (int e = 0; e < kPer; e += 2) *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
-    if (lane == 0) a.lse[r] = mx + logf(wsum);
+      for (int j = 0; j < kRows; ++j) {
+        mxj[j] = __shfl_sync(0xffffffffu, mx, (j0 + j) & 31);
+        invj[j] = __shfl_sync(0xffffffffu, inv, (j0 + j) & 31);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[j][e] = 0.f;
+      }
+#pragma unroll 2
+      for (int s = 0; s < S; ++s) {
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) {
+          const long long r = r0 + j0 + j;
+          if (j0 + j < nr && FA_IN(kSiteCombine, (long long)s * rows + r, 1, (long long)S * rows, a.err)) {
+            const float ls = a.part_lse[(long long)s * rows + r];
+            const float w = ls == -INFINITY ? 0.f : __expf(ls - mxj[j]);
+            const float* src = a.part_o + ((long long)s * rows + r) * D + lane * kPer;
+            if constexpr (kPer == 4) {
+              const float4 v = *reinterpret_cast<const float4*>(src);
+              acc[j][0] += w * v.x, acc[j][1] += w * v.y, acc[j][2] += w * v.z, acc[j][3] += w * v.w;
+            } else {
+              const float2 v = *reinterpret_cast<const float2*>(src);
+              acc[j][0] += w * v.x, acc[j][1] += w * v.y;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        if (j0 + j >= nr) continue;
+        const long long r = r0 + j0 + j;
+        const int bh = (int)(r / a.N), i = (int)(r - (long long)bh * a.N);
+        const int b_ = bh / a.H, h_ = bh - b_ * a.H;
+        const long long ooff = b_ * a.o_sb + h_ * a.o_sh + (long long)i * a.o_sn;
+        if (!FA_IN(kSiteCombine, ooff, D, o_lim, a.err)) continue;
+        __nv_bfloat16* orow = a.o + ooff + lane * kPer;
+        if constexpr (kPer == 4)
+          *reinterpret_cast<uint2*>(orow) = make_uint2(pack_bf16x2(acc[j][0] * invj[j], acc[j][1] * invj[j]),
+                                                       pack_bf16x2(acc[j][2] * invj[j], acc[j][3] * invj[j]));
+        else
+          *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(acc[j][0] * invj[j], acc[j][1] * invj[j]);
+      }
+    }
   }
 }
 

@@ -211,3 +211,40 @@ def test_one_rank_nccl_group_runs_the_cuda_orchestration(cuda_device, tmp_path):
             parity.check("dV", dv, rdv)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("B,H,N,d,S", [(2, 3, 130, 64, 1), (2, 3, 130, 128, 3), (2, 3, 130, 64, 40),
+                                        (2, 3, 130, 128, 8), (3, 2, 6667, 128, 3), (3, 5, 20500, 64, 2)])
+def test_merge_partials_against_its_definition(cuda_device, B, H, N, d, S):
+    """fa_merge_partials on random pieces and logsumexps, some -inf and one
+    row -inf in every piece, against the definition in fp64: lse = ln sum_s
+    e^lse_s, O = sum_s e^(lse_s - lse) O_s rounded to bf16; O = 0 and
+    lse = -inf where nothing is seen.  The kernel's grid (1184 blocks of 8
+    warps) takes rows in groups of G per warp, G the largest power of two up
+    to 32 with G x 9472 <= rows: G = 1 for 780 rows, 4 for 40002 and 32 for
+    307500 rows, the last two ending in a partial group."""
+    g = torch.Generator().manual_seed(100 + d + S + N)
+    all_lse = torch.randn((S, B, H, N), generator=g, dtype=torch.float64) * 6
+    all_lse[torch.rand((S, B, H, N), generator=g) < 0.3] = float("-inf")
+    all_lse[:, 0, 1, 9] = float("-inf")
+    all_lse[0, 1, 1, 3] = 5.0  # one piece alone: O is that piece
+    all_lse[1:, 1, 1, 3] = float("-inf")
+    all_lse = all_lse.float().double()
+    pieces = torch.randn((S, B, H, N, d), generator=g, dtype=torch.float64).float().double()
+    o, lse = binding.merge_partials(pieces.float().to(cuda_device).contiguous(),
+                                    all_lse.float().to(cuda_device).contiguous())
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    ref_lse = torch.logsumexp(all_lse, dim=0)
+    w = torch.nan_to_num(torch.exp(all_lse - ref_lse), nan=0.0)
+    ref = (w[..., None] * pieces).sum(0)
+    got = o.double().cpu()
+    # bf16 output: half an ulp (at most 2^-8 of |O|) plus the fp32 sum of up to
+    # 40 weighted terms of magnitude < 5 (2e-5)
+    assert ((got - ref).abs() <= ref.abs() * 2 ** -8 + 2e-5).all(), (got - ref).abs().max().item()
+    assert torch.equal(got[0, 1, 9], torch.zeros(d, dtype=torch.float64))
+    assert torch.equal(got[1, 1, 3], pieces[0, 1, 1, 3].float().bfloat16().double())
+    lc = lse.double().cpu()
+    fin = torch.isfinite(ref_lse)
+    assert torch.equal(torch.isneginf(lc), ~fin)
+    assert ((lc[fin] - ref_lse[fin]).abs() <= 1e-5 + 1e-7 * ref_lse[fin].abs()).all()
