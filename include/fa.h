@@ -311,10 +311,13 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
  *   a row whose pieces are all -inf gets 0 and lse -inf.  The sum of the
  *   weighted pieces over the parts (an all-reduce) is O in fp32;
  *   fa_merge_partials with num_parts = 1 on that sum and lse converts it to
- *   bf16.  part_o 16-byte aligned, all_lse and lse 4-byte aligned
- *   (FA_ERR_ALIGNMENT); 1 <= num_parts <= 4096 and 0 <= part < num_parts
- *   (FA_ERR_INVALID_ARG); a failed launch returns FA_ERR_CUDA without
- *   updating fa_last_cuda_error (cudaGetLastError has the code).
+ *   bf16.  d in {64, 128} (FA_ERR_UNSUPPORTED); part_o 16-byte aligned,
+ *   all_lse and lse 4-byte aligned (FA_ERR_ALIGNMENT); 1 <= num_parts <=
+ *   4096 and 0 <= part < num_parts (FA_ERR_INVALID_ARG); B*H*N*num_parts
+ *   above 2^40 gives FA_ERR_TOO_LARGE; an empty problem returns FA_OK and
+ *   launches nothing.  Asynchronous on `stream`.  A failed launch returns
+ *   FA_ERR_CUDA without updating fa_last_cuda_error (cudaGetLastError has
+ *   the code).
  * fa_bwd_recompute_range: the recompute stage of fa_bwd for the window's
  *   keys: writes dk, dv of those keys (complete) and adds their part of dQ
  *   into the workspace's fp32 accumulator.  Run fa_bwd_prepare (on the full

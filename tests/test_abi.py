@@ -234,3 +234,5 @@ def test_weight_partial_arguments_are_rejected_before_launch(lib):
     assert w(po=24) == binding.FA_ERR_ALIGNMENT and w(al=18) == binding.FA_ERR_ALIGNMENT
     assert w(lse=18) == binding.FA_ERR_ALIGNMENT
     assert w(B=0) == binding.FA_OK and w(B=-1) == binding.FA_ERR_INVALID_ARG  # empty: nothing launched
+    # B*H*N*num_parts = 2^30 * 2 * 100 * 4096 > 2^40 is refused before any launch
+    assert lib.fa_weight_partial(16, 16, 4096, 0, 16, 1 << 30, 2, 100, 64, None) == binding.FA_ERR_TOO_LARGE
