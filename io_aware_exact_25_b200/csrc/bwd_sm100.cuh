@@ -299,15 +299,16 @@ struct BwdLayout {
   // issue, TMA producer, two idle warps) so that every warpgroup is whole for
   // the register reallocation: launched at 128 registers a thread (the whole
   // register file), then for the P/dS warpgroups, dQ and warpgroup 3
-  // 152 / 112 / 88 without dropout and 160 / 104 / 80 with it (both sum to
-  // 2*128*R_ps + 128*R_dq + 128*R_ctl = 64512 <= 65536).  At 128 registers
-  // for every warp the dropout kernels spilled 220-280 bytes a thread; with
-  // these splits none of the kernels without dropout spills (the long8k
-  // backward 1.7 % faster than at 160/104/80, which spilled 48 bytes) and the
-  // dropout kernels spill 0-12 (160/112/72 spills 4 there but measured 1 %
-  // slower on long64k).
+  // 152 / 112 / 88 without dropout, 160 / 112 / 80 with it at d = 128 and
+  // 160 / 104 / 80 with it at d = 64 (2*128*R_ps + 128*R_dq + 128*R_ctl =
+  // 64512, 65536 and 64512 <= 65536).  At 128 registers for every warp the
+  // dropout kernels spilled 220-280 bytes a thread; with these splits no
+  // kernel spills (ptxas).  Without dropout the long8k backward is 1.7 %
+  // faster than at 160/104/80, which spilled 48 bytes; at d = 128 with
+  // dropout 160/104/80 spilled 12-16 bytes and 160/112/72 4, and 160/112/80
+  // spills none at d = 128 but 4-28 bytes at d = 64.
   static constexpr int kThreads = 512;
-  static constexpr uint32_t kRegsPS = DROPOUT ? 160 : 152, kRegsDQ = DROPOUT ? 104 : 112,
+  static constexpr uint32_t kRegsPS = DROPOUT ? 160 : 152, kRegsDQ = DROPOUT ? (D == 128 ? 112 : 104) : 112,
                             kRegsCtl = DROPOUT ? 80 : 88;
   static_assert(2 * 128 * kRegsPS + 128 * kRegsDQ + 128 * kRegsCtl <= 512 * 128, "register split");
   static constexpr uint32_t kHalf = 128u * 128u;
